@@ -1,0 +1,161 @@
+"""B200 (sm_100a) fused exact attention forward — Python binding.
+
+A thin ctypes layer over the C ABI in ``include/attn.h`` (the in-tree library
+``libattn_b200.so``). It only marshals arguments: it checks dtypes, devices and
+contiguity, allocates outputs with torch, and passes raw pointers and the
+current CUDA stream. Every step of the computation runs in the library's CUDA
+kernels; there is no other implementation to fall back to — if the library is
+missing or cannot run, the call raises.
+
+    o, lse = attn_fwd(q, k, v, causal=True)          # bf16 [B,H,N,d] on cuda
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libattn_b200.so")
+
+STATUS_NAMES = {
+    0: "ATTN_OK",
+    1: "ATTN_ERR_INVALID_ARG",
+    2: "ATTN_ERR_UNSUPPORTED",
+    3: "ATTN_ERR_ALIGNMENT",
+    4: "ATTN_ERR_CUDA",
+    5: "ATTN_ERR_TIMEOUT",
+    6: "ATTN_ERR_WORKSPACE",
+}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+_lib = None
+_lock = threading.Lock()
+
+_c_int, _c_float, _vp, _sz = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+_SIGNATURES = {
+    "attn_fwd": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp]),
+    "attn_fwd_host_buffer_size": (_sz, [_c_int] * 6),
+    "attn_fwd_host": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp, _sz, _vp]),
+    "attn_get_status": (_c_int, [_vp]),
+    "attn_get_status_ex": (_c_int, [_vp, ctypes.POINTER(_c_int)]),
+    "attn_set_timeout_ms": (_c_int, [_c_int]),
+    "attn_status_string": (ctypes.c_char_p, [_c_int]),
+    "attn_version": (_c_int, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load (once) and return the C library; raises if it was never built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"CUDA library not built: {LIB_PATH} is missing "
+                    "(run `python -m exact_attention_134_b200.build`)")
+            l = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in _SIGNATURES.items():
+                fn = getattr(l, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = l
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise AttnError(status, what)
+
+
+def _stream_handle(device=None) -> int:
+    import torch
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _shape_args(q, k, v):
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, N, d]")
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nkv, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk != d:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)} k {tuple(k.shape)} v {tuple(v.shape)}")
+    return B, Hq, Hkv, Nq, Nkv, d
+
+
+def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None):
+    """Fused exact attention forward on the GPU.
+
+    q: bf16 cuda [B, Hq, Nq, d]; k, v: bf16 cuda [B, Hkv, Nkv, d] (contiguous).
+    Returns (o bf16 [B, Hq, Nq, d], lse fp32 [B, Hq, Nq]) with
+    lse = ln sum_j exp(scale * q.k_j) (scale defaults to 1/sqrt(d)).
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    B, Hq, Hkv, Nq, Nkv, d = _shape_args(q, k, v)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    st = lib().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                        B, Hq, Hkv, Nq, Nkv, d, int(bool(causal)), float(scale),
+                        _stream_handle(q.device))
+    _check(st, "attn_fwd")
+    return out, lse
+
+
+def host_buffer_size(B, Hq, Hkv, Nq, Nkv, d) -> int:
+    return int(lib().attn_fwd_host_buffer_size(B, Hq, Hkv, Nq, Nkv, d))
+
+
+def attn_fwd_host(q, k, v, causal: bool = False, scale: float | None = None, dev_buf=None,
+                  out=None, lse=None):
+    """Same operation on HOST (CPU, ideally pinned) bf16 tensors: the library
+    copies inputs to the device buffer ``dev_buf`` (a uint8 cuda tensor of at
+    least ``host_buffer_size`` bytes; allocated here if None), computes, copies
+    O and LSE back and synchronises. Returns CPU tensors (o, lse)."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CPU tensor")
+    B, Hq, Hkv, Nq, Nkv, d = _shape_args(q, k, v)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = host_buffer_size(B, Hq, Hkv, Nq, Nkv, d)
+    if dev_buf is None:
+        dev_buf = torch.empty(need, dtype=torch.uint8, device="cuda")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32)
+    st = lib().attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                             B, Hq, Hkv, Nq, Nkv, d, int(bool(causal)), float(scale),
+                             dev_buf.data_ptr(), dev_buf.numel(), _stream_handle(dev_buf.device))
+    _check(st, "attn_fwd_host")
+    return out, lse
+
+
+def get_status(stream: int | None = None) -> tuple[int, int]:
+    """Synchronise the stream and return (status, where) from the device status word."""
+    where = ctypes.c_int(0)
+    s = lib().attn_get_status_ex(_stream_handle() if stream is None else stream, ctypes.byref(where))
+    return int(s), int(where.value)
+
+
+def set_timeout_ms(ms: int):
+    _check(lib().attn_set_timeout_ms(int(ms)), "attn_set_timeout_ms")
+
+
+def version() -> int:
+    return int(lib().attn_version())

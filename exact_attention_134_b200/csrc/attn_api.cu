@@ -1,0 +1,212 @@
+// attn_api.cu — the C ABI declared in include/attn.h: argument validation,
+// tensor-map (TMA descriptor) construction, launch, device status word.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "attn_internal.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Device status word: [0] = attn_status_t code of the first failure since the
+// last read, [1] = where it happened (role / tile, for diagnostics).
+__device__ int g_status[4];
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+std::mutex g_dev_mutex;
+int* g_status_ptr[kMaxDevices] = {nullptr};
+std::atomic<long long> g_timeout_ns{1000000000LL};
+
+void load_encode() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                       &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+}
+
+// Per-device one-time set-up with that device current: the driver's tensor-map
+// encoder and the device address of the status word.
+int* device_status_ptr() {
+  std::call_once(g_encode_once, load_encode);
+  if (!g_encode) return nullptr;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (!g_status_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(ptr);
+  }
+  return g_status_ptr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+attn_status_t check_args(const void* q, const void* k, const void* v, const void* o,
+                         const void* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                         int causal, float scale) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nkv <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.0f)) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (causal && Nq != Nkv) return ATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || Hq > 65535) return ATTN_ERR_UNSUPPORTED;
+  // TMA global strides must stay below 2^40 bytes.
+  const unsigned long long head_bytes_q = 2ull * (unsigned long long)Nq * d;
+  const unsigned long long head_bytes_kv = 2ull * (unsigned long long)Nkv * d;
+  if (head_bytes_q >= (1ull << 40) || head_bytes_kv >= (1ull << 40)) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_ALIGNMENT;
+  return ATTN_OK;
+}
+
+// bf16 tensor [BH, N, d] as a 3-D map {d, N, BH}; box = 64 columns x 128 rows,
+// 128-byte swizzle (the layout the tcgen05 descriptors expect).
+bool make_map(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * (cuuint64_t)d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t elem_strides[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                        strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
+                      cudaStream_t stream) {
+  int* status = device_status_ptr();
+  if (!status) return ATTN_ERR_CUDA;
+  alignas(64) CUtensorMap tq, tk, tv, to;
+  if (!make_map(&tq, q, d, Nq, (long long)B * Hq) || !make_map(&tk, k, d, Nkv, (long long)B * Hkv) ||
+      !make_map(&tv, v, d, Nkv, (long long)B * Hkv) || !make_map(&to, o, d, Nq, (long long)B * Hq))
+    return ATTN_ERR_CUDA;
+  attn_sm100::FwdParams p;
+  p.lse = lse;
+  p.status = status;
+  p.Nq = Nq;
+  p.Nkv = Nkv;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.causal = causal;
+  const int rows = attn_sm100::fwd_rows_per_cta();
+  p.num_row_blocks = (Nq + rows - 1) / rows;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = (unsigned long long)g_timeout_ns.load();
+  cudaError_t e = attn_sm100::launch_fwd_bf16(tq, tk, tv, to, p, B, Hq, d, stream);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct HostLayout {
+  size_t q, k, v, o, lse, total;
+};
+
+HostLayout host_layout(int B, int Hq, int Hkv, int Nq, int Nkv, int d) {
+  HostLayout L;
+  const size_t qo = 2ull * B * Hq * (size_t)Nq * d;
+  const size_t kv = 2ull * B * Hkv * (size_t)Nkv * d;
+  L.q = 0;
+  L.k = round_up(L.q + qo, 256);
+  L.v = round_up(L.k + kv, 256);
+  L.o = round_up(L.v + kv, 256);
+  L.lse = round_up(L.o + qo, 256);
+  L.total = round_up(L.lse + 4ull * B * Hq * (size_t)Nq, 256);
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
+                       void* stream) {
+  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  if (s != ATTN_OK) return s;
+  return run_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale,
+                 static_cast<cudaStream_t>(stream));
+}
+
+size_t attn_fwd_host_buffer_size(int B, int Hq, int Hkv, int Nq, int Nkv, int d) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nkv <= 0 || d <= 0) return 0;
+  return host_layout(B, Hq, Hkv, Nq, Nkv, d).total;
+}
+
+attn_status_t attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                            void* o_host, float* lse_host, int B, int Hq, int Hkv, int Nq, int Nkv,
+                            int d, int causal, float scale, void* dev_buf, size_t dev_buf_bytes,
+                            void* stream) {
+  attn_status_t s =
+      check_args(q_host, k_host, v_host, o_host, lse_host, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  if (s != ATTN_OK) return s;
+  if (!dev_buf || !aligned16(dev_buf)) return ATTN_ERR_WORKSPACE;
+  const HostLayout L = host_layout(B, Hq, Hkv, Nq, Nkv, d);
+  if (dev_buf_bytes < L.total) return ATTN_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(dev_buf);
+  const size_t qo = 2ull * B * Hq * (size_t)Nq * d;
+  const size_t kv = 2ull * B * Hkv * (size_t)Nkv * d;
+  if (cudaMemcpyAsync(base + L.q, q_host, qo, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(base + L.k, k_host, kv, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(base + L.v, v_host, kv, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  s = run_fwd(base + L.q, base + L.k, base + L.v, base + L.o, reinterpret_cast<float*>(base + L.lse),
+              B, Hq, Hkv, Nq, Nkv, d, causal, scale, st);
+  if (s != ATTN_OK) return s;
+  if (cudaMemcpyAsync(o_host, base + L.o, qo, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(lse_host, base + L.lse, 4ull * B * Hq * (size_t)Nq, cudaMemcpyDeviceToHost,
+                      st) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return cudaStreamSynchronize(st) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_get_status_ex(void* stream, int* where) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  int h[2] = {0, 0};
+  if (cudaMemcpyFromSymbol(h, g_status, sizeof(h)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (where) *where = h[1];
+  if (h[0] != 0) {
+    const int zero[2] = {0, 0};
+    if (cudaMemcpyToSymbol(g_status, zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return static_cast<attn_status_t>(h[0]);
+}
+
+attn_status_t attn_get_status(void* stream) { return attn_get_status_ex(stream, nullptr); }
+
+attn_status_t attn_set_timeout_ms(int ms) {
+  if (ms < 1) return ATTN_ERR_INVALID_ARG;
+  g_timeout_ns.store((long long)ms * 1000000LL);
+  return ATTN_OK;
+}
+
+const char* attn_status_string(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_ALIGNMENT: return "ATTN_ERR_ALIGNMENT";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE";
+  }
+  return "ATTN_ERR_UNKNOWN";
+}
+
+int attn_version(void) { return 100; }
+
+}  // extern "C"

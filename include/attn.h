@@ -1,0 +1,116 @@
+/*
+ * attn.h — C ABI of the B200 (sm_100a) fused exact-attention forward.
+ *
+ * Operation (the definition on "FlashAttention (TR)", systems-analysis.info,
+ * section "Standart Attention Mekanizmasının Sorunları"):
+ *     O = softmax(scale * Q K^T [+ causal mask]) V,
+ *     LSE_i = ln sum_j exp(scale * (Q K^T)_ij)   over the keys row i sees,
+ * computed the fused way the same page describes in "Tiling ve Blok Tabanlı
+ * İşleme", "Çevrimiçi Softmax Hesaplama" and "İşlemlerin Tek Bir CUDA
+ * Çekirdeğinde Birleştirilmesi": K/V tiles streamed through on-chip memory,
+ * a running row maximum and exponential sum, one kernel, only O and LSE
+ * written to HBM (no N x N matrix is ever stored).
+ *
+ * Conventions shared by every entry point
+ *   - Layout: Q and O are contiguous bf16 [B, Hq, Nq, d]; K and V contiguous
+ *     bf16 [B, Hkv, Nkv, d]; LSE contiguous fp32 [B, Hq, Nq] (natural log,
+ *     scale included).
+ *   - GQA: query head h reads kv head h / (Hq / Hkv) (contiguous groups; the
+ *     pages name MQA only, "FlashAttention-2 (2023)" section). Hq % Hkv == 0.
+ *   - Causal: key j is visible to query i iff j <= i; requires Nq == Nkv.
+ *   - Head dim d is 64 or 128.
+ *   - Ownership: the caller owns every buffer; device pointers must stay valid
+ *     until the work queued on `stream` has finished. The library allocates no
+ *     device memory. `stream` is a cudaStream_t (0 = legacy default stream).
+ *   - Asynchrony: work is queued on `stream`; nothing synchronises except
+ *     where an entry point says so.
+ *   - Errors: the return value is the only channel (nothing is printed, no
+ *     exception crosses the ABI). Arguments are validated before anything is
+ *     queued; a rejected call leaves every buffer untouched. Device-side
+ *     failures (a pipeline wait that exceeded its time budget) are recorded in
+ *     a device status word that attn_get_status() reads.
+ *   - Alignment: every device pointer must be 16-byte aligned (tensor-memory
+ *     accelerator descriptors require it); else ATTN_ERR_ALIGNMENT.
+ */
+#ifndef EXACT_ATTENTION_134_B200_ATTN_H
+#define EXACT_ATTENTION_134_B200_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,  /* NULL pointer, a size <= 0, Hq % Hkv != 0, scale not finite or <= 0 */
+  ATTN_ERR_UNSUPPORTED = 2,  /* d not in {64, 128}; causal with Nq != Nkv; sizes beyond 2^31 elements per tensor dim */
+  ATTN_ERR_ALIGNMENT = 3,    /* a device pointer is not 16-byte aligned */
+  ATTN_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (no device, launch failure, ...) */
+  ATTN_ERR_TIMEOUT = 5,      /* a kernel pipeline wait exceeded its budget (reported by attn_get_status) */
+  ATTN_ERR_WORKSPACE = 6     /* workspace pointer NULL/misaligned or smaller than the required size */
+} attn_status_t;
+
+/*
+ * attn_fwd — bf16 fused exact attention forward.
+ *   q      device, bf16 [B, Hq, Nq, d]          (read)
+ *   k, v   device, bf16 [B, Hkv, Nkv, d]        (read)
+ *   o      device, bf16 [B, Hq, Nq, d]          (written; RNE from fp32)
+ *   lse    device, fp32 [B, Hq, Nq]             (written)
+ *   scale  softmax scale applied to Q K^T (typically 1/sqrt(d)); finite, > 0
+ *   causal 0 = full attention, 1 = lower-triangular mask (needs Nq == Nkv)
+ * Allocates nothing; one kernel launch on `stream`.
+ */
+ATTN_API attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                       int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                       int causal, float scale, void* stream);
+
+/*
+ * attn_fwd_host — the same operation on HOST buffers, for callers whose data
+ * lives in host memory. Copies q, k, v into `dev_buf` (a device buffer of at
+ * least attn_fwd_host_buffer_size() bytes, 16-byte aligned, owned by the
+ * caller), runs attn_fwd on `stream`, copies o and lse back and synchronises
+ * `stream` before returning. Host buffers should be page-locked for the copies
+ * to run at full speed (pageable memory works, slower).
+ */
+ATTN_API size_t attn_fwd_host_buffer_size(int B, int Hq, int Hkv, int Nq, int Nkv, int d);
+ATTN_API attn_status_t attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                            void* o_host, float* lse_host,
+                            int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                            int causal, float scale,
+                            void* dev_buf, size_t dev_buf_bytes, void* stream);
+
+/*
+ * attn_get_status — synchronises `stream`, returns and clears the device
+ * status word (ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel gave up on a pipeline
+ * wait since the last call). Returns ATTN_ERR_CUDA if synchronisation fails.
+ */
+ATTN_API attn_status_t attn_get_status(void* stream);
+
+/* attn_get_status_ex — as attn_get_status; also stores in *where (if not
+ * NULL) a diagnostic code naming the kernel role and tile that gave up
+ * (0 when nothing failed). */
+ATTN_API attn_status_t attn_get_status_ex(void* stream, int* where);
+
+/* attn_set_timeout_ms — budget of every in-kernel pipeline wait (default 1000
+ * ms; values < 1 are rejected with ATTN_ERR_INVALID_ARG). Process-wide. */
+ATTN_API attn_status_t attn_set_timeout_ms(int ms);
+
+/* Human-readable name of a status code (static storage). */
+ATTN_API const char* attn_status_string(attn_status_t status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+ATTN_API int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTENTION_134_B200_ATTN_H */

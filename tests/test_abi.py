@@ -1,0 +1,82 @@
+"""C-ABI checks that need no GPU: the library builds and loads, exports every
+entry point include/attn.h declares, and rejects bad arguments before it
+touches CUDA (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_attention_134_b200 as attn
+from exact_attention_134_b200 import build as attn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    attn_build.build()
+    return attn.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_symbols()
+    assert "attn_fwd" in names and len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_strings(lib):
+    assert attn.version() >= 100
+    assert lib.attn_status_string(0) == b"ATTN_OK"
+    assert lib.attn_status_string(5) == b"ATTN_ERR_TIMEOUT"
+    assert lib.attn_status_string(99) == b"ATTN_ERR_UNKNOWN"
+
+
+P = 0x10000  # a fake, 16-byte-aligned "device pointer": never dereferenced on these paths
+
+
+def _fwd(lib, q=P, k=P, v=P, o=P, lse=P, B=1, Hq=2, Hkv=2, Nq=128, Nkv=128, d=128, causal=0, scale=0.125):
+    return lib.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), 1), (dict(lse=0), 1), (dict(B=0), 1), (dict(Nq=0), 1), (dict(Nkv=-1), 1),
+    (dict(Hq=3, Hkv=2), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1),
+    (dict(scale=float("inf")), 1), (dict(scale=-1.0), 1), (dict(causal=2), 1),
+    (dict(d=96), 2), (dict(d=256), 2), (dict(causal=1, Nq=128, Nkv=256), 2),
+    (dict(q=P + 2), 3), (dict(o=P + 8), 3), (dict(lse=P + 4), 3),
+])
+def test_argument_validation(lib, kw, code):
+    assert _fwd(lib, **kw) == code
+
+
+def test_host_entry_rejects_bad_workspace(lib):
+    need = lib.attn_fwd_host_buffer_size(1, 2, 2, 128, 128, 64)
+    assert need >= 2 * (2 * 128 * 64 * 2) + 2 * 128 * 64 * 2 + 2 * 128 * 4
+    args = [P, P, P, P, P, 1, 2, 2, 128, 128, 64, 0, 0.125]
+    assert lib.attn_fwd_host(*args, None, need, None) == 6
+    assert lib.attn_fwd_host(*args, P + 1, need, None) == 6
+    assert lib.attn_fwd_host(*args, P, need - 1, None) == 6
+    assert lib.attn_fwd_host_buffer_size(0, 2, 2, 128, 128, 64) == 0
+
+
+def test_timeout_setter(lib):
+    assert lib.attn_set_timeout_ms(0) == 1
+    assert lib.attn_set_timeout_ms(1000) == 0
+
+
+def test_binding_requires_cuda_tensors():
+    import torch
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        attn.attn_fwd(q, q, q)
