@@ -293,10 +293,14 @@ def run_ours(args):
     ms = res["total_ms"] / args.steps
     value = world * w.flops / (ms * 1e-3) / 1e12
     per_launch_tflops = w.flops / (statistics.mean(res["times"]) * 1e-3) / 1e12
-    e2e_ms, h2d, d2h = bench_e2e(w, max(2, args.steps // 2), 1, world, rank, attn)
-    e2e_value = world * w.flops / (e2e_ms / max(2, args.steps // 2) * 1e-3) / 1e12
+    e2e = None
+    if not args.kernel_only:
+        e2e_steps = max(2, args.steps // 2)
+        e2e_ms, h2d, d2h = bench_e2e(w, e2e_steps, 1, world, rank, attn)
+        e2e = {"value": round(world * w.flops / (e2e_ms / e2e_steps * 1e-3) / 1e12, 2),
+               "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     extras = {}
-    if not args.no_extra:
+    if not args.no_extra and not args.kernel_only:
         for name in EXTRA_BF16:
             if name == args.workload:
                 continue
@@ -311,7 +315,9 @@ def run_ours(args):
             torch.cuda.empty_cache()
     out = None
     if rank == 0:
-        cpu = cpu_baseline(w, *res["inputs"], budget_s=args.cpu_budget) if world == 1 else None
+        cpu = None
+        if world == 1 and not args.kernel_only:
+            cpu = cpu_baseline(w, *res["inputs"], budget_s=args.cpu_budget)
         traffic = _traffic_from_profile(args.workload)
         out = {
             "metric": METRIC,
@@ -337,8 +343,7 @@ def run_ours(args):
                          "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
                          "kernel": "attn_fwd_bf16_kernel",
                          "algorithmic_min_bytes": w.min_hbm_bytes},
-            "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+            "e2e": e2e,
             "gpu_launches": args.steps,
             "clocks": clk,
             "cpu_baseline": cpu,
@@ -392,6 +397,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true", help="skip the other bf16 workloads")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="only the device-timed leg (for profiling runs): no e2e, CPU or extra legs")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

@@ -137,14 +137,23 @@ def test_no_writes_outside_outputs():
 
 
 def test_non_default_scale_and_stream():
+    # scale 0.3 (3.4x 1/sqrt(128)) makes rows peaky: a few keys dominate, so the
+    # bf16 rounding of P (relative error up to 2^-8 per weight) no longer
+    # averages out. The bound per output is that rounding applied to every
+    # term, 2^-8 * sum_j P_ij |V_jc|, plus half a bf16 ulp for rounding O.
     q, k, v = make_qkv(1, 2, 2, 333, 333, 128, seed=9)
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
         o, lse = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True, scale=0.3)
     s.synchronize()
-    O, L = oracle.attention_fp64(bf16_bits(q), bf16_bits(k), bf16_bits(v), True, 0.3)
-    mx, mean, dl = _compare(o.cpu(), lse.cpu(), O, L)
-    assert mx <= MAX_TOL and mean <= MEAN_TOL and dl <= LSE_TOL
+    O, L, P = oracle.attention_fp64(bf16_bits(q), bf16_bits(k), bf16_bits(v), True, 0.3, return_p=True)
+    og = o.cpu().float().numpy().astype(np.float64)
+    vabs = np.abs(oracle.widen_bf16(bf16_bits(v)))
+    p_bound = 2.0 ** -8 * np.einsum("bhij,bhjc->bhic", P, vabs)
+    half_ulp = 2.0 ** (np.floor(np.log2(np.abs(O) + p_bound + 1e-30)) - 8)
+    assert np.all(np.abs(og - O) <= p_bound + half_ulp + 1e-4)
+    assert np.abs(og - O).mean() <= MEAN_TOL
+    assert np.abs(lse.cpu().numpy() - L).max() <= LSE_TOL
 
 
 def test_host_buffer_entry_point():
