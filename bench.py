@@ -222,6 +222,36 @@ def bench_workload(w: Workload, steps: int, warmup: int, world: int, rank: int, 
             "flops": w.flops}
 
 
+def bench_q8(w: Workload, steps: int, warmup: int, world: int, rank: int, lib_mod):
+    """8-bit path: time of the whole call (3 prepass launches + main kernel) and
+    of the prepass alone; the main kernel's share is the difference."""
+    import torch
+    wr = rank_workload(w, rank)
+    q, k, v = make_qkv(wr.B, wr.Hq, wr.Hkv, wr.Nq, wr.Nkv, wr.d, wr.seed, wr.dist)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o = torch.empty_like(qd)
+    lse = torch.empty((wr.B, wr.Hq, wr.Nq), dtype=torch.float32, device="cuda")
+    ws = torch.empty(lib_mod.q8_workspace_size(wr.B, wr.Hq, wr.Hkv, wr.Nq, wr.Nkv, wr.d),
+                     dtype=torch.uint8, device="cuda")
+
+    def full():
+        lib_mod.attn_fwd_q8(qd, kd, vd, causal=w.causal, workspace=ws, out=o, lse=lse)
+
+    def pre():
+        lib_mod.q8_prepass(qd, kd, vd, ws)
+
+    _barrier(world)
+    t_full = time_device(full, steps, max(warmup, 3))
+    t_pre = time_device(pre, steps, 3)
+    _barrier(world)
+    st, where = lib_mod.get_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} at {where:#x}")
+    full_ms = _max_over_ranks(statistics.mean(t_full), world)
+    pre_ms = _max_over_ranks(statistics.mean(t_pre), world)
+    return full_ms, pre_ms
+
+
 def bench_e2e(w: Workload, steps: int, warmup: int, world: int, rank: int, lib_mod):
     """Same metric through the host-buffer entry point: every step copies the
     step's inputs from pinned host memory and reads O and LSE back."""
@@ -313,6 +343,18 @@ def run_ours(args):
                             "l2": r["l2"]}
             del r
             torch.cuda.empty_cache()
+        wq = WORKLOADS["q8_8k_outlier"]
+        full_ms, pre_ms = bench_q8(wq, max(3, args.steps // 2), 3, world, rank, attn)
+        fp8_peak = 2.0 * peaks["bf16"]
+        extras["q8_8k_outlier"] = {
+            "tflops": round(world * wq.flops / (full_ms * 1e-3) / 1e12, 1),
+            "ms_per_step": round(full_ms, 4), "prepass_ms": round(pre_ms, 4),
+            "main_ms": round(full_ms - pre_ms, 4),
+            "main_tflops": round(world * wq.flops / ((full_ms - pre_ms) * 1e-3) / 1e12, 1),
+            "frac_of_fp8_peak_main": round(wq.flops / ((full_ms - pre_ms) * 1e-3) / 1e12 / fp8_peak, 4),
+            "fp8_peak": f"{fp8_peak:.0f} TFLOP/s = 2 x measured bf16 (nominal fp8/bf16 ratio)",
+            "l2": "inputs_larger_than_l2"}
+        torch.cuda.empty_cache()
     out = None
     if rank == 0:
         cpu = None

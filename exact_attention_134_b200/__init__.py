@@ -44,6 +44,10 @@ _SIGNATURES = {
     "attn_fwd": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp]),
     "attn_fwd_host_buffer_size": (_sz, [_c_int] * 6),
     "attn_fwd_host": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp, _sz, _vp]),
+    "attn_fwd_q8_workspace_size": (_sz, [_c_int] * 6),
+    "attn_fwd_q8": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp, _sz, _vp]),
+    "attn_q8_prepass": (_c_int, [_vp, _vp, _vp] + [_c_int] * 6 + [_vp, _sz, _vp]),
+    "attn_q8_workspace_offsets": (_c_int, [_c_int] * 6 + [ctypes.POINTER(_sz)]),
     "attn_get_status": (_c_int, [_vp]),
     "attn_get_status_ex": (_c_int, [_vp, ctypes.POINTER(_c_int)]),
     "attn_set_timeout_ms": (_c_int, [_c_int]),
@@ -113,6 +117,54 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None
                         _stream_handle(q.device))
     _check(st, "attn_fwd")
     return out, lse
+
+
+def q8_workspace_size(B, Hq, Hkv, Nq, Nkv, d) -> int:
+    return int(lib().attn_fwd_q8_workspace_size(B, Hq, Hkv, Nq, Nkv, d))
+
+
+def q8_workspace_offsets(B, Hq, Hkv, Nq, Nkv, d) -> list[int]:
+    """Byte offsets of the 8-bit workspace regions (q8, k8, v8, sq, sk, sv,
+    kbar, qk, K partial sums, V partial maxima) and the total size."""
+    arr = (_sz * 11)()
+    _check(lib().attn_q8_workspace_offsets(B, Hq, Hkv, Nq, Nkv, d, arr), "attn_q8_workspace_offsets")
+    return [int(x) for x in arr]
+
+
+def attn_fwd_q8(q, k, v, causal: bool = False, scale: float | None = None, workspace=None,
+                out=None, lse=None):
+    """8-bit (INT8 Q K^T after K smoothing, FP8 P V) attention forward.
+
+    Same tensors as ``attn_fwd``; ``workspace`` is a uint8 cuda tensor of at
+    least ``q8_workspace_size`` bytes (allocated here if None). Returns (o, lse).
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    B, Hq, Hkv, Nq, Nkv, d = _shape_args(q, k, v)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if workspace is None:
+        workspace = torch.empty(q8_workspace_size(B, Hq, Hkv, Nq, Nkv, d), dtype=torch.uint8,
+                                device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    st = lib().attn_fwd_q8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                           B, Hq, Hkv, Nq, Nkv, d, int(bool(causal)), float(scale),
+                           workspace.data_ptr(), workspace.numel(), _stream_handle(q.device))
+    _check(st, "attn_fwd_q8")
+    return out, lse
+
+
+def q8_prepass(q, k, v, workspace):
+    """Run only the 8-bit prepass (K mean, scales, quantisation) into ``workspace``."""
+    B, Hq, Hkv, Nq, Nkv, d = _shape_args(q, k, v)
+    st = lib().attn_q8_prepass(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, Nq, Nkv, d,
+                               workspace.data_ptr(), workspace.numel(), _stream_handle(q.device))
+    _check(st, "attn_q8_prepass")
 
 
 def host_buffer_size(B, Hq, Hkv, Nq, Nkv, d) -> int:

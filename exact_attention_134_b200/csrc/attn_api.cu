@@ -84,6 +84,19 @@ bool make_map(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
   return r == CUDA_SUCCESS;
 }
 
+// 8-bit tensor [BH, N, d] as {d, N, BH}; box = d bytes x 128 rows, swizzle = d bytes.
+bool make_map_u8(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)N * (cuuint64_t)d};
+  cuuint32_t box[3] = {(cuuint32_t)d, 128, 1};
+  cuuint32_t elem_strides[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides,
+                        box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                       int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
                       cudaStream_t stream) {
@@ -110,6 +123,80 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace of the 8-bit path, in this order, each region 256-byte aligned:
+// q8, k8, v8 (1 byte per element), sq, sk, sv, kbar, qk (fp32), ksum partials
+// (fp64), vmax partials (fp32).
+constexpr int kQ8Regions = 10;
+
+void q8_layout(int B, int Hq, int Hkv, int Nq, int Nkv, int d, size_t off[kQ8Regions + 1]) {
+  const size_t nqb = (size_t)(Nq + 127) / 128, nkb = (size_t)(Nkv + 127) / 128;
+  const size_t sz[kQ8Regions] = {
+      (size_t)B * Hq * Nq * d,      (size_t)B * Hkv * Nkv * d,   (size_t)B * Hkv * Nkv * d,
+      4ull * B * Hq * nqb,          4ull * B * Hkv * nkb,        4ull * B * Hkv * d,
+      4ull * B * Hkv * d,           4ull * B * Hq * (size_t)Nq,  8ull * B * Hkv * nkb * d,
+      4ull * B * Hkv * nkb * d};
+  size_t o = 0;
+  for (int i = 0; i < kQ8Regions; ++i) {
+    off[i] = o;
+    o = round_up(o + sz[i], 256);
+  }
+  off[kQ8Regions] = o;
+}
+
+attn_status_t run_q8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
+                     void* workspace, size_t workspace_bytes, bool prepass_only,
+                     cudaStream_t stream) {
+  if (!workspace || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
+  size_t off[kQ8Regions + 1];
+  q8_layout(B, Hq, Hkv, Nq, Nkv, d, off);
+  if (workspace_bytes < off[kQ8Regions]) return ATTN_ERR_WORKSPACE;
+  int* status = device_status_ptr();
+  if (!status) return ATTN_ERR_CUDA;
+  char* w = static_cast<char*>(workspace);
+  attn_sm100::Q8Launch L;
+  std::memset(static_cast<void*>(&L), 0, sizeof(L));
+  L.q = q;
+  L.k = k;
+  L.v = v;
+  L.q8 = reinterpret_cast<int8_t*>(w + off[0]);
+  L.k8 = reinterpret_cast<int8_t*>(w + off[1]);
+  L.v8 = reinterpret_cast<uint8_t*>(w + off[2]);
+  L.kbar = reinterpret_cast<float*>(w + off[6]);
+  L.ksum_part = reinterpret_cast<double*>(w + off[8]);
+  L.vmax_part = reinterpret_cast<float*>(w + off[9]);
+  L.B = B;
+  L.Hkv = Hkv;
+  L.prepass_only = prepass_only;
+  attn_sm100::Q8Params& p = L.p;
+  p.lse = lse;
+  p.status = status;
+  p.sq = reinterpret_cast<const float*>(w + off[3]);
+  p.sk = reinterpret_cast<const float*>(w + off[4]);
+  p.sv = reinterpret_cast<const float*>(w + off[5]);
+  p.qk = reinterpret_cast<const float*>(w + off[7]);
+  p.Nq = Nq;
+  p.Nkv = Nkv;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.causal = causal;
+  p.num_row_blocks = (Nq + 255) / 256;
+  p.nqb = (Nq + 127) / 128;
+  p.nkb = (Nkv + 127) / 128;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale = scale;
+  p.timeout_ns = (unsigned long long)g_timeout_ns.load();
+  if (!prepass_only) {
+    if (!make_map_u8(&L.tq, L.q8, d, Nq, (long long)B * Hq) ||
+        !make_map_u8(&L.tk, L.k8, d, Nkv, (long long)B * Hkv) ||
+        !make_map_u8(&L.tv, L.v8, d, Nkv, (long long)B * Hkv) ||
+        !make_map(&L.to, o, d, Nq, (long long)B * Hq))
+      return ATTN_ERR_CUDA;
+  }
+  cudaError_t e = attn_sm100::launch_q8(L, d, stream);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
 
 struct HostLayout {
   size_t q, k, v, o, lse, total;
@@ -172,6 +259,42 @@ attn_status_t attn_fwd_host(const void* q_host, const void* k_host, const void* 
                       st) != cudaSuccess)
     return ATTN_ERR_CUDA;
   return cudaStreamSynchronize(st) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t attn_fwd_q8_workspace_size(int B, int Hq, int Hkv, int Nq, int Nkv, int d) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nkv <= 0 || d <= 0) return 0;
+  size_t off[kQ8Regions + 1];
+  q8_layout(B, Hq, Hkv, Nq, Nkv, d, off);
+  return off[kQ8Regions];
+}
+
+attn_status_t attn_q8_workspace_offsets(int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                                        size_t* offsets) {
+  if (!offsets || B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nkv <= 0 || d <= 0)
+    return ATTN_ERR_INVALID_ARG;
+  size_t off[kQ8Regions + 1];
+  q8_layout(B, Hq, Hkv, Nq, Nkv, d, off);
+  for (int i = 0; i <= kQ8Regions; ++i) offsets[i] = off[i];
+  return ATTN_OK;
+}
+
+attn_status_t attn_fwd_q8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                          int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  if (s != ATTN_OK) return s;
+  return run_q8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, workspace,
+                workspace_bytes, false, static_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_q8_prepass(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
+                              int Nq, int Nkv, int d, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  // o / lse are not touched by the prepass; reuse the common checks with q in their place
+  attn_status_t s = check_args(q, k, v, q, q, B, Hq, Hkv, Nq, Nkv, d, 0, 1.0f);
+  if (s != ATTN_OK) return s;
+  return run_q8(q, k, v, nullptr, nullptr, B, Hq, Hkv, Nq, Nkv, d, 0, 1.0f, workspace,
+                workspace_bytes, true, static_cast<cudaStream_t>(stream));
 }
 
 attn_status_t attn_get_status_ex(void* stream, int* where) {

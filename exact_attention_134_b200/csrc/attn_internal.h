@@ -21,6 +21,42 @@ struct FwdParams {
   unsigned long long timeout_ns;  // budget of every pipeline wait
 };
 
+// Kernel parameters of the 8-bit main kernel.
+struct Q8Params {
+  float* lse;                     // fp32 [B, Hq, Nq]
+  int* status;                    // device status word
+  const float* sq;                // [B, Hq, nqb]   Q block scales
+  const float* sk;                // [B, Hkv, nkb]  smoothed-K block scales
+  const float* sv;                // [B, Hkv, d]    V channel scales
+  const float* qk;                // [B, Hq, Nq]    q_i . kbar
+  int Nq, Nkv, Hq, Hkv;
+  int causal;
+  int num_row_blocks;
+  int nqb, nkb;                   // 128-token blocks of Q and K/V
+  float scale_log2;               // scale * log2(e)
+  float scale;
+  unsigned long long timeout_ns;
+};
+
+// Everything one 8-bit forward needs (prepass + main kernel).
+struct Q8Launch {
+  CUtensorMap tq, tk, tv, to;     // over q8, k8, v8 (uint8) and o (bf16)
+  Q8Params p;
+  const void* q;                  // bf16 inputs
+  const void* k;
+  const void* v;
+  int8_t* q8;
+  int8_t* k8;
+  uint8_t* v8;
+  float* kbar;
+  double* ksum_part;
+  float* vmax_part;
+  int B, Hkv;
+  bool prepass_only;
+};
+
+cudaError_t launch_q8(const Q8Launch& L, int d, cudaStream_t stream);
+
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& to, const FwdParams& p, int B, int Hq, int d,
                             cudaStream_t stream);

@@ -1,0 +1,653 @@
+// attn_q8_sm100.cu — 8-bit attention forward in the manner of the page
+// "Makale Bülteni — SageAttention" (section "İddia ve Gerçeklik:
+// SageAttention"): the first GEMM (Q K^T) runs on INT8 tensor cores after K is
+// mean-centred ("smoothing" — lossless, softmax is shift invariant), the
+// second (P V) on FP8 because P already lies in [0, 1]; accumulation stays in
+// fp32.
+//
+// Steps (one stream, four launches):
+//   1. kv_stats   per 128-token chunk: fp64 partial sums of K (per channel),
+//                 partial max |V| (per channel)
+//   2. kv_final   K channel mean kbar (fp64 sum / Nkv, rounded once to fp32),
+//                 V channel scale sv = max|V| / 448
+//   3. quantize   Q -> INT8, one fp32 scale per 128-token block, plus
+//                 qk_i = q_i . kbar (to undo the smoothing shift in LSE);
+//                 K - kbar -> INT8 per 128-token block; V / sv -> e4m3
+//   4. main       the fused forward: S = Q8 K8^T (kind::i8, s32 in TMEM),
+//                 online softmax on s * sq * sk * scale, P -> e4m3(p * 448)
+//                 written back to TMEM, O += P8 V8 (kind::f8f6f4, fp32 in
+//                 TMEM), O = O * sv / (448 l), LSE += scale * qk.
+// Every quantisation decision (scale, code) is taken in fp32 with correctly
+// rounded division and round-half-even, so the codes are reproducible.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "attn_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace attn_sm100 {
+
+namespace {
+
+constexpr int kQ8Threads = 320;
+constexpr int kTok = 128;         // tokens per quantisation block == MMA tile rows
+constexpr int kPrepThreads = 256;
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+  f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x);
+  f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+  f[4] = bf16_lo(u.z); f[5] = bf16_hi(u.z);
+  f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
+}
+
+__device__ __forceinline__ int8_t quant_i8(float x, float s) {
+  int c = __float2int_rn(__fdiv_rn(x, s));  // round half to even
+  c = c > 127 ? 127 : (c < -127 ? -127 : c);
+  return static_cast<int8_t>(c);
+}
+
+// Block-wide max of non-negative floats (256 threads).
+__device__ __forceinline__ float block_max256(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float m = red[0];
+#pragma unroll
+  for (int i = 1; i < kPrepThreads / 32; ++i) m = fmaxf(m, red[i]);
+  return m;
+}
+
+// ----------------------------------------------------------------- prepass 1
+template <int D>
+__global__ void __launch_bounds__(kPrepThreads)
+    q8_kv_stats_kernel(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, int Nkv,
+                       int nkb, double* __restrict__ ksum_part, float* __restrict__ vmax_part) {
+  constexpr int VPR = D / 8;              // 16-byte vectors per row
+  constexpr int RPP = kPrepThreads / VPR;  // rows per pass
+  __shared__ double ssum[RPP][D];
+  __shared__ float smax[RPP][D];
+  const int tid = threadIdx.x, vc = tid % VPR, rs = tid / VPR;
+  const size_t bh = (size_t)blockIdx.z * gridDim.y + blockIdx.y;
+  const int t0 = blockIdx.x * kTok;
+  double s[8];
+  float mx[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) { s[i] = 0.0; mx[i] = 0.0f; }
+  for (int r = rs; r < kTok; r += RPP) {
+    const int t = t0 + r;
+    if (t >= Nkv) break;
+    const size_t off = (bh * Nkv + t) * D + vc * 8;
+    float kf[8], vf[8];
+    unpack8(*reinterpret_cast<const uint4*>(k + off), kf);
+    unpack8(*reinterpret_cast<const uint4*>(v + off), vf);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      s[i] += static_cast<double>(kf[i]);
+      mx[i] = fmaxf(mx[i], fabsf(vf[i]));
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    ssum[rs][vc * 8 + i] = s[i];
+    smax[rs][vc * 8 + i] = mx[i];
+  }
+  __syncthreads();
+  if (tid < D) {
+    double acc = 0.0;
+    float m = 0.0f;
+    for (int r = 0; r < RPP; ++r) {
+      acc += ssum[r][tid];
+      m = fmaxf(m, smax[r][tid]);
+    }
+    ksum_part[(bh * nkb + blockIdx.x) * D + tid] = acc;
+    vmax_part[(bh * nkb + blockIdx.x) * D + tid] = m;
+  }
+}
+
+// ----------------------------------------------------------------- prepass 2
+template <int D>
+__global__ void q8_kv_final_kernel(const double* __restrict__ ksum_part,
+                                   const float* __restrict__ vmax_part, int Nkv, int nkb,
+                                   float* __restrict__ kbar, float* __restrict__ sv) {
+  const size_t bh = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+  const int c = threadIdx.x;
+  double acc = 0.0;
+  float m = 0.0f;
+  for (int i = 0; i < nkb; ++i) {
+    acc += ksum_part[(bh * nkb + i) * D + c];
+    m = fmaxf(m, vmax_part[(bh * nkb + i) * D + c]);
+  }
+  kbar[bh * D + c] = static_cast<float>(acc / static_cast<double>(Nkv));
+  sv[bh * D + c] = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
+}
+
+// ----------------------------------------------------------------- prepass 3
+template <int D>
+__global__ void __launch_bounds__(kPrepThreads)
+    q8_quantize_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                       const uint16_t* __restrict__ v, int B, int Hq, int Hkv, int Nq, int Nkv,
+                       int nqb, int nkb, const float* __restrict__ kbar,
+                       const float* __restrict__ sv, int8_t* __restrict__ q8,
+                       int8_t* __restrict__ k8, uint8_t* __restrict__ v8, float* __restrict__ sq,
+                       float* __restrict__ sk, float* __restrict__ qk) {
+  constexpr int VPR = D / 8;
+  constexpr int RPP = kPrepThreads / VPR;
+  constexpr int NP = kTok / RPP;  // passes
+  __shared__ float red[kPrepThreads / 32];
+  const int tid = threadIdx.x, vc = tid % VPR, rs = tid / VPR;
+  const long long n_q_tiles = (long long)B * Hq * nqb;
+  long long tile = blockIdx.x;
+  float x[NP][8];
+  if (tile < n_q_tiles) {
+    const int qb = (int)(tile % nqb);
+    const long long bh = tile / nqb;  // b * Hq + h
+    const int b = (int)(bh / Hq), h = (int)(bh % Hq);
+    const size_t bhk = (size_t)b * Hkv + h / (Hq / Hkv);
+    float amax = 0.0f;
+#pragma unroll
+    for (int pp = 0; pp < NP; ++pp) {
+      const int t = qb * kTok + rs + pp * RPP;
+      if (t < Nq) {
+        unpack8(*reinterpret_cast<const uint4*>(q + ((size_t)bh * Nq + t) * D + vc * 8), x[pp]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[pp][i] = 0.0f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[pp][i]));
+    }
+    amax = block_max256(amax, red);
+    const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 1.0f;
+    float kb[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) kb[i] = kbar[bhk * D + vc * 8 + i];
+#pragma unroll
+    for (int pp = 0; pp < NP; ++pp) {
+      const int t = qb * kTok + rs + pp * RPP;
+      float dot = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dot = fmaf(x[pp][i], kb[i], dot);
+#pragma unroll
+      for (int o = VPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      if (t < Nq) {
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          lo |= (uint32_t)(uint8_t)quant_i8(x[pp][i], s) << (8 * i);
+          hi |= (uint32_t)(uint8_t)quant_i8(x[pp][i + 4], s) << (8 * i);
+        }
+        *reinterpret_cast<uint2*>(q8 + ((size_t)bh * Nq + t) * D + vc * 8) = make_uint2(lo, hi);
+        if (vc == 0) qk[(size_t)bh * Nq + t] = dot;
+      }
+    }
+    if (tid == 0) sq[(size_t)bh * nqb + qb] = s;
+  } else {
+    tile -= n_q_tiles;
+    const int kb_i = (int)(tile % nkb);
+    const size_t bh = (size_t)(tile / nkb);  // b * Hkv + h
+    float kb[8], svc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      kb[i] = kbar[bh * D + vc * 8 + i];
+      svc[i] = sv[bh * D + vc * 8 + i];
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int pp = 0; pp < NP; ++pp) {
+      const int t = kb_i * kTok + rs + pp * RPP;
+      if (t < Nkv) {
+        unpack8(*reinterpret_cast<const uint4*>(k + (bh * Nkv + t) * D + vc * 8), x[pp]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[pp][i] = x[pp][i] - kb[i];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[pp][i] = 0.0f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[pp][i]));
+    }
+    amax = block_max256(amax, red);
+    const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 1.0f;
+#pragma unroll
+    for (int pp = 0; pp < NP; ++pp) {
+      const int t = kb_i * kTok + rs + pp * RPP;
+      if (t < Nkv) {
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          lo |= (uint32_t)(uint8_t)quant_i8(x[pp][i], s) << (8 * i);
+          hi |= (uint32_t)(uint8_t)quant_i8(x[pp][i + 4], s) << (8 * i);
+        }
+        *reinterpret_cast<uint2*>(k8 + (bh * Nkv + t) * D + vc * 8) = make_uint2(lo, hi);
+        float vf[8];
+        unpack8(*reinterpret_cast<const uint4*>(v + (bh * Nkv + t) * D + vc * 8), vf);
+        uint32_t w0 = pack_e4m3x2(__fdiv_rn(vf[0], svc[0]), __fdiv_rn(vf[1], svc[1])) |
+                      (pack_e4m3x2(__fdiv_rn(vf[2], svc[2]), __fdiv_rn(vf[3], svc[3])) << 16);
+        uint32_t w1 = pack_e4m3x2(__fdiv_rn(vf[4], svc[4]), __fdiv_rn(vf[5], svc[5])) |
+                      (pack_e4m3x2(__fdiv_rn(vf[6], svc[6]), __fdiv_rn(vf[7], svc[7])) << 16);
+        *reinterpret_cast<uint2*>(v8 + (bh * Nkv + t) * D + vc * 8) = make_uint2(w0, w1);
+      }
+    }
+    if (tid == 0) sk[bh * nkb + kb_i] = s;
+  }
+}
+
+// ----------------------------------------------------------------- main kernel
+template <int D>
+struct Q8Cfg {
+  static constexpr int kTileBytes = kTok * D;  // 8-bit tile: 128 rows x D bytes
+  static constexpr int kStages = 8;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffRing = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
+  static constexpr int kOffSv = kOffBar + 512;
+  static constexpr int kSmemBytes = kOffBar + 1024 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128;
+  static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
+  static constexpr int kOutBoxBytes = 128 * 128;  // bf16 output box: 128 rows x 64 columns
+};
+
+struct Q8Bar {
+  static constexpr int kFull = 0, kEmpty = 8, kQFull = 16, kSFull = 17, kPFull = 19,
+                       kOFinal = 21, kEpi = 22, kDrain = 24;
+  static constexpr int kTmemSlotByte = 8 * 32;
+  static constexpr int kAbortByte = 8 * 32 + 4;
+};
+
+__device__ __forceinline__ void q8_flag_abort(volatile int* abort_flag, int* status, int where) {
+  *abort_flag = 1;
+  if (atomicCAS(status, 0, ATTN_ERR_TIMEOUT) == 0) status[1] = where;
+}
+
+__device__ __forceinline__ bool q8_warp_all(bool v) { return __all_sync(0xffffffffu, v) != 0; }
+
+template <int D>
+__device__ __forceinline__ void issue_qk_i8(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+  constexpr uint32_t idesc = idesc_s8_s32(128, 128);
+#pragma unroll
+  for (int kk = 0; kk < D / 32; ++kk) {
+    const uint64_t a = smem_desc_sw(q_smem + kk * 32, 16, 8 * D, D);
+    const uint64_t b = smem_desc_sw(k_smem + kk * 32, 16, 8 * D, D);
+    mma_i8_ss(d_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv_f8(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem,
+                                            bool accumulate) {
+  constexpr uint32_t idesc = idesc_e4m3_f32_bmn(128, D);
+#pragma unroll
+  for (int kk = 0; kk < kTok / 32; ++kk) {
+    const uint64_t b = smem_desc_sw(v_smem + kk * 32 * D, kTok * D, 8 * D, D);
+    mma_f8_ts(o_tmem, p_tmem + kk * 8, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kQ8Threads, 1)
+    attn_fwd_q8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                       const Q8Params p) {
+  using C = Q8Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_addr(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - raw_base);
+  const uint32_t sQ = base + C::kOffQ;
+  const uint32_t sRing = base + C::kOffRing;
+  const uint32_t sBar = base + C::kOffBar;
+  auto bar = [&](int slot) -> uint32_t { return sBar + 8u * slot; };
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kOffBar + Q8Bar::kTmemSlotByte);
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kOffBar + Q8Bar::kAbortByte);
+  float* const sv_smem = reinterpret_cast<float*>(base_ptr + C::kOffSv);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int row_block = p.causal ? (p.num_row_blocks - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+  const int hq = blockIdx.y, b = blockIdx.z;
+  const int hk = hq / (p.Hq / p.Hkv);
+  const int q0 = row_block * 2 * kTok;
+  const int bh_q = b * p.Hq + hq;
+  const int bh_kv = b * p.Hkv + hk;
+  int n_tiles;
+  if (p.causal) {
+    const int last_row = min(q0 + 2 * kTok - 1, p.Nq - 1);
+    n_tiles = min(last_row, p.Nkv - 1) / kTok + 1;
+  } else {
+    n_tiles = (p.Nkv + kTok - 1) / kTok;
+  }
+  const uint64_t budget = p.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar(Q8Bar::kFull + s), 1);
+      mbar_init(bar(Q8Bar::kEmpty + s), 1);
+    }
+    mbar_init(bar(Q8Bar::kQFull), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(Q8Bar::kSFull + t), 1);
+      mbar_init(bar(Q8Bar::kPFull + t), 128);
+      mbar_init(bar(Q8Bar::kEpi + t), 128);
+    }
+    mbar_init(bar(Q8Bar::kOFinal), 1);
+    mbar_init(bar(Q8Bar::kDrain), 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (threadIdx.x < D) sv_smem[threadIdx.x] = p.sv[(size_t)bh_kv * D + threadIdx.x];
+  if (warp == 8) {
+    tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 9 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer
+    bool ok = true;
+    uint32_t issued = 0;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(Q8Bar::kQFull), 2 * C::kTileBytes);
+      for (int t = 0; t < 2; ++t)
+        tma_load_3d(sQ + t * C::kTileBytes, &tm_q, bar(Q8Bar::kQFull), 0, q0 + t * kTok, bh_q);
+    }
+    for (int j = 0; j < n_tiles && ok; ++j) {
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t stage = issued % C::kStages;
+        const uint32_t phase = (issued / C::kStages) & 1u;
+        ok = q8_warp_all(bounded_wait(bar(Q8Bar::kEmpty + stage), phase ^ 1u, abort_flag, budget));
+        if (!ok) break;
+        if (lane == 0) {
+          const uint32_t fb = bar(Q8Bar::kFull + stage);
+          mbar_arrive_expect_tx(fb, C::kTileBytes);
+          tma_load_3d(sRing + stage * C::kTileBytes, which ? &tm_v : &tm_k, fb, 0, j * kTok, bh_kv);
+        }
+        __syncwarp();
+        ++issued;
+      }
+    }
+    if (!ok) {
+      if (lane == 0) {
+        q8_flag_abort(abort_flag, p.status, 0x1100);
+        volatile int no_abort = 0;
+        bounded_wait(bar(Q8Bar::kQFull), 0, &no_abort, budget);
+        const uint32_t first = issued > (uint32_t)C::kStages ? issued - C::kStages : 0u;
+        for (uint32_t i = first; i < issued; ++i)
+          bounded_wait(bar(Q8Bar::kFull + i % C::kStages), (i / C::kStages) & 1u, &no_abort, budget);
+      }
+      __syncwarp();
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t tS[2] = {tmem + C::kColS0, tmem + C::kColS1};
+    const uint32_t tO[2] = {tmem + C::kColO0, tmem + C::kColO1};
+    const uint32_t q_smem[2] = {sQ, sQ + C::kTileBytes};
+    bool ok = q8_warp_all(bounded_wait(bar(Q8Bar::kQFull), 0, abort_flag, budget));
+    uint32_t slot = 0, v_prev_stage = 0;
+    int j = 0;
+    for (; j < n_tiles && ok; ++j) {
+      const uint32_t k_stage = slot % C::kStages, k_phase = (slot / C::kStages) & 1u;
+      ++slot;
+      const uint32_t v_stage = slot % C::kStages;
+      ++slot;
+      const uint32_t k_smem = sRing + k_stage * C::kTileBytes;
+      ok = q8_warp_all(bounded_wait(bar(Q8Bar::kFull + k_stage), k_phase, abort_flag, budget));
+      if (!ok) break;
+      if (j > 0) {
+        const uint32_t vp_slot = slot - 3;
+        ok = q8_warp_all(bounded_wait(bar(Q8Bar::kPFull + 0), (j - 1) & 1, abort_flag, budget) &&
+                         bounded_wait(bar(Q8Bar::kFull + v_prev_stage), (vp_slot / C::kStages) & 1u,
+                                      abort_flag, budget));
+        if (!ok) break;
+        tc_fence_after();
+        if (lane == 0) issue_pv_f8<D>(tO[0], tS[0], sRing + v_prev_stage * C::kTileBytes, j - 1 > 0);
+      }
+      tc_fence_after();
+      if (lane == 0) {
+        issue_qk_i8<D>(tS[0], q_smem[0], k_smem);
+        tc_commit(bar(Q8Bar::kSFull + 0));
+      }
+      __syncwarp();
+      if (j > 0) {
+        ok = q8_warp_all(bounded_wait(bar(Q8Bar::kPFull + 1), (j - 1) & 1, abort_flag, budget));
+        if (!ok) break;
+        tc_fence_after();
+        if (lane == 0) {
+          issue_pv_f8<D>(tO[1], tS[1], sRing + v_prev_stage * C::kTileBytes, j - 1 > 0);
+          tc_commit(bar(Q8Bar::kEmpty + v_prev_stage));
+        }
+      }
+      if (lane == 0) {
+        issue_qk_i8<D>(tS[1], q_smem[1], k_smem);
+        tc_commit(bar(Q8Bar::kSFull + 1));
+        tc_commit(bar(Q8Bar::kEmpty + k_stage));
+      }
+      __syncwarp();
+      v_prev_stage = v_stage;
+    }
+    if (ok) {
+      const int jl = n_tiles - 1;
+      const uint32_t vp_slot = slot - 1;
+      ok = q8_warp_all(bounded_wait(bar(Q8Bar::kPFull + 0), jl & 1, abort_flag, budget) &&
+                       bounded_wait(bar(Q8Bar::kFull + v_prev_stage), (vp_slot / C::kStages) & 1u,
+                                    abort_flag, budget));
+      if (ok) {
+        tc_fence_after();
+        if (lane == 0) issue_pv_f8<D>(tO[0], tS[0], sRing + v_prev_stage * C::kTileBytes, jl > 0);
+        __syncwarp();
+        ok = q8_warp_all(bounded_wait(bar(Q8Bar::kPFull + 1), jl & 1, abort_flag, budget));
+        if (ok) {
+          tc_fence_after();
+          if (lane == 0) {
+            issue_pv_f8<D>(tO[1], tS[1], sRing + v_prev_stage * C::kTileBytes, jl > 0);
+            tc_commit(bar(Q8Bar::kEmpty + v_prev_stage));
+            tc_commit(bar(Q8Bar::kOFinal));
+          }
+          __syncwarp();
+        }
+      }
+    }
+    if (!ok) {
+      if (lane == 0) {
+        q8_flag_abort(abort_flag, p.status, 0x1200 | (j << 12));
+        tc_commit(bar(Q8Bar::kDrain));
+        volatile int no_abort = 0;
+        bounded_wait(bar(Q8Bar::kDrain), 0, &no_abort, budget);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int t = warp >> 2;
+    const int wq = warp & 3;
+    const int r = (wq << 5) | lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq << 5) << 16;
+    const uint32_t tS = tmem + (t ? C::kColS1 : C::kColS0) + lane_off;
+    const uint32_t tO = tmem + (t ? C::kColO1 : C::kColO0) + lane_off;
+    const int row = q0 + t * kTok + r;
+    const int qtile = (q0 >> 7) + t;
+    // a tile wholly past Nq has no scale; its rows are computed but never stored
+    const float sq_t = qtile < p.nqb ? p.sq[(size_t)bh_q * p.nqb + qtile] : 1.0f;
+    const float kLog2_448 = 8.807354922057604f;  // log2(448)
+
+    float m_run = -INFINITY;  // running maximum of scale*log2(e)*S (exact: rescale on every increase)
+    float l_run = 0.0f;       // sum of 448 * 2^(. - m_run)
+    bool ok = true;
+    int j = 0;
+    for (; j < n_tiles; ++j) {
+      ok = q8_warp_all(bounded_wait(bar(Q8Bar::kSFull + t), j & 1, abort_flag, budget));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+      tmem_wait_ld();
+      const float f = sq_t * p.sk[(size_t)bh_kv * p.nkb + j] * p.scale_log2;
+      const int kv0 = j * kTok;
+      int lim = p.Nkv - kv0;
+      if (p.causal) lim = min(lim, row - kv0 + 1);
+#pragma unroll
+      for (int c = 0; c < kTok; ++c) {
+        const float sf = static_cast<float>(static_cast<int>(sr[c]));
+        sr[c] = __float_as_uint(c < lim ? sf : -INFINITY);
+      }
+      float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
+      float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
+#pragma unroll
+      for (int c = 4; c < kTok; c += 4) {
+        mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
+        mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+        mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
+        mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
+      }
+      // f > 0 (all scales positive), so the max of s*f is f * max(s)
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * f;
+      float alpha = 1.0f;
+      if (m_tile > m_run) {
+        alpha = ex2_approx(m_run - m_tile);
+        m_run = m_tile;
+      }
+      const float mb = (m_run == -INFINITY) ? 0.0f : m_run;
+      const float bias = kLog2_448 - mb;  // p448 = 448 * 2^(s*f - m) = 2^(s*f - m + log2 448)
+      float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < kTok; c += 4) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c]), f, bias));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), f, bias));
+        const float p2 = ex2_approx(fmaf(__uint_as_float(sr[c + 2]), f, bias));
+        const float p3 = ex2_approx(fmaf(__uint_as_float(sr[c + 3]), f, bias));
+        sum0 += p0 + p2;
+        sum1 += p1 + p3;
+        sr[c >> 2] = pack_e4m3x2(p0, p1) | (pack_e4m3x2(p2, p3) << 16);
+      }
+      tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&sr[0]));
+      const bool rescale = (j > 0) && (alpha != 1.0f);
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + 32 * c, o);
+        }
+      }
+      l_run = l_run * alpha + (sum0 + sum1);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(Q8Bar::kPFull + t));
+    }
+
+    if (ok) ok = q8_warp_all(bounded_wait(bar(Q8Bar::kOFinal), 0, abort_flag, budget));
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+      // The K/V ring is idle once every MMA has completed; stage the bf16 O
+      // tile of query tile t in it (32 KiB at d = 128).
+      uint8_t* const stage_ptr = base_ptr + C::kOffRing + t * (D / 64) * C::kOutBoxBytes;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * c, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) {
+          const int col16 = c * 4 + qd;
+          const int bx = col16 >> 3;
+          const int ch = col16 & 7;
+          float y[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            y[i] = __uint_as_float(o[8 * qd + i]) * sv_smem[col16 * 8 + i] * inv_l;
+          uint4 v;
+          v.x = pack_bf16x2(y[0], y[1]);
+          v.y = pack_bf16x2(y[2], y[3]);
+          v.z = pack_bf16x2(y[4], y[5]);
+          v.w = pack_bf16x2(y[6], y[7]);
+          *reinterpret_cast<uint4*>(stage_ptr + bx * C::kOutBoxBytes + r * 128 + ((ch ^ (r & 7)) << 4)) = v;
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(Q8Bar::kEpi + t));
+      if (row < p.Nq) {
+        // l_run carries the factor 448, which O's numerator also carries
+        const float lse2 = m_run + log2f(l_run) - kLog2_448;
+        p.lse[(size_t)bh_q * p.Nq + row] =
+            lse2 * 0.69314718055994530942f + p.scale * p.qk[(size_t)bh_q * p.Nq + row];
+      }
+      if (r == 0) {
+        volatile int no_abort = 0;
+        if (bounded_wait(bar(Q8Bar::kEpi + t), 0, &no_abort, budget)) {
+          for (int bx = 0; bx < D / 64; ++bx)
+            tma_store_3d(&tm_o, smem_addr(stage_ptr) + bx * C::kOutBoxBytes, bx * 64, q0 + t * kTok, bh_q);
+          tma_store_commit();
+          tma_store_wait_all();
+        } else {
+          q8_flag_abort(abort_flag, p.status, 0x1400 | t);
+        }
+      }
+    } else if (lane == 0) {
+      q8_flag_abort(abort_flag, p.status, 0x1300 | (t << 8) | (j << 12));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch_q8_d(const Q8Launch& L, cudaStream_t stream) {
+  const int nqb = L.p.nqb, nkb = L.p.nkb;
+  dim3 g1(nkb, L.Hkv, L.B);
+  q8_kv_stats_kernel<D><<<g1, kPrepThreads, 0, stream>>>(
+      static_cast<const uint16_t*>(L.k), static_cast<const uint16_t*>(L.v), L.p.Nkv, nkb,
+      L.ksum_part, L.vmax_part);
+  dim3 g2(L.Hkv, L.B);
+  q8_kv_final_kernel<D><<<g2, D, 0, stream>>>(L.ksum_part, L.vmax_part, L.p.Nkv, nkb, L.kbar,
+                                              const_cast<float*>(L.p.sv));
+  const long long tiles = (long long)L.B * L.p.Hq * nqb + (long long)L.B * L.Hkv * nkb;
+  q8_quantize_kernel<D><<<(unsigned)tiles, kPrepThreads, 0, stream>>>(
+      static_cast<const uint16_t*>(L.q), static_cast<const uint16_t*>(L.k),
+      static_cast<const uint16_t*>(L.v), L.B, L.p.Hq, L.Hkv, L.p.Nq, L.p.Nkv, nqb, nkb, L.kbar,
+      L.p.sv, L.q8, L.k8, L.v8, const_cast<float*>(L.p.sq), const_cast<float*>(L.p.sk),
+      const_cast<float*>(L.p.qk));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || L.prepass_only) return e;
+  e = cudaFuncSetAttribute(attn_fwd_q8_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Q8Cfg<D>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(L.p.num_row_blocks, L.p.Hq, L.B);
+  attn_fwd_q8_kernel<D><<<grid, kQ8Threads, Q8Cfg<D>::kSmemBytes, stream>>>(L.tq, L.tk, L.tv, L.to, L.p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_q8(const Q8Launch& L, int d, cudaStream_t stream) {
+  return d == 128 ? launch_q8_d<128>(L, stream) : launch_q8_d<64>(L, stream);
+}
+
+}  // namespace attn_sm100

@@ -88,6 +88,51 @@ ATTN_API attn_status_t attn_fwd_host(const void* q_host, const void* k_host, con
                             void* dev_buf, size_t dev_buf_bytes, void* stream);
 
 /*
+ * attn_fwd_q8 — the same operation through the 8-bit mainloop of
+ * "Makale Bülteni — SageAttention" (section "İddia ve Gerçeklik:
+ * SageAttention"): K is mean-centred per (batch, kv head, channel) over all
+ * Nkv tokens (lossless by the shift invariance of softmax; LSE is corrected
+ * back), Q and the smoothed K are quantised to INT8 with one fp32 scale per
+ * 128-token block, V to FP8 e4m3 with one fp32 scale per channel; S = Q8 K8^T
+ * runs on INT8 tensor cores (s32 accumulation), P is encoded as e4m3(p * 448)
+ * and P8 V8 runs on FP8 tensor cores (fp32 accumulation).
+ *   inputs/outputs  as attn_fwd (bf16 q, k, v; bf16 o; fp32 lse)
+ *   workspace       device, caller-owned, 16-byte aligned, at least
+ *                   attn_fwd_q8_workspace_size() bytes; holds the quantised
+ *                   tensors and scales (its contents after the call are the
+ *                   prepass results, see attn_q8_workspace_offsets)
+ * Four launches on `stream` (three prepass kernels, one main kernel).
+ * Errors: as attn_fwd, plus ATTN_ERR_WORKSPACE for a NULL, misaligned or too
+ * small workspace.
+ */
+ATTN_API size_t attn_fwd_q8_workspace_size(int B, int Hq, int Hkv, int Nq, int Nkv, int d);
+ATTN_API attn_status_t attn_fwd_q8(const void* q, const void* k, const void* v, void* o, float* lse,
+                                   int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                                   int causal, float scale,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_q8_prepass — only the three prepass launches of attn_fwd_q8 (K mean,
+ * V channel scales, quantisation of Q, K, V), writing the workspace; used to
+ * time the prepass on its own and to inspect its results.
+ */
+ATTN_API attn_status_t attn_q8_prepass(const void* q, const void* k, const void* v,
+                                       int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_q8_workspace_offsets — byte offsets of the workspace regions, in
+ * order: q8 int8 [B,Hq,Nq,d], k8 int8 [B,Hkv,Nkv,d] (smoothed), v8 e4m3
+ * [B,Hkv,Nkv,d], sq fp32 [B,Hq,ceil(Nq/128)], sk fp32 [B,Hkv,ceil(Nkv/128)],
+ * sv fp32 [B,Hkv,d], kbar fp32 [B,Hkv,d], qk fp32 [B,Hq,Nq] (q_i . kbar),
+ * K partial sums fp64 [B,Hkv,ceil(Nkv/128),d], V partial maxima fp32
+ * [B,Hkv,ceil(Nkv/128),d]; offsets[10] = total size. `offsets` holds 11
+ * entries.
+ */
+ATTN_API attn_status_t attn_q8_workspace_offsets(int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                                                 size_t* offsets);
+
+/*
  * attn_get_status — synchronises `stream`, returns and clears the device
  * status word (ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel gave up on a pipeline
  * wait since the last call). Returns ATTN_ERR_CUDA if synchronisation fails.

@@ -80,3 +80,20 @@ def test_binding_requires_cuda_tensors():
     q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         attn.attn_fwd(q, q, q)
+
+
+def test_q8_entry_validation(lib):
+    need = lib.attn_fwd_q8_workspace_size(1, 2, 2, 300, 300, 128)
+    off = (ctypes.c_size_t * 11)()
+    assert lib.attn_q8_workspace_offsets(1, 2, 2, 300, 300, 128, off) == 0
+    assert off[10] == need and list(off) == sorted(off)
+    assert all(o % 256 == 0 for o in off)
+    # q8 / k8 / v8 hold one byte per element, then the fp32 scales
+    assert off[1] - off[0] >= 2 * 300 * 128 and off[3] - off[2] >= 2 * 300 * 128
+    args = [P, P, P, P, P, 1, 2, 2, 300, 300, 128, 0, 0.125]
+    assert lib.attn_fwd_q8(*args, None, need, None) == 6
+    assert lib.attn_fwd_q8(*args, P + 8, need, None) == 6
+    assert lib.attn_fwd_q8(*args, P, need - 1, None) == 6
+    assert lib.attn_fwd_q8(P, P, P, P, P, 1, 2, 2, 300, 300, 96, 0, 0.125, P, need, None) == 2
+    assert lib.attn_q8_prepass(P, P, P, 1, 2, 2, 300, 300, 128, None, need, None) == 6
+    assert lib.attn_q8_workspace_offsets(0, 2, 2, 300, 300, 128, off) == 1

@@ -1,0 +1,132 @@
+"""GPU parity of the 8-bit (SageAttention-style) path.
+
+Prepass: the quantised codes and scales are compared bit for bit with the
+oracle's 8-bit steps (both sides decide every code in fp32 with correctly
+rounded division and round-half-even); q.kbar within fp32 rounding.
+
+Forward: against the EXACT fp64 oracle (not the quantised one) with the 8-bit
+tolerance: cosine >= 0.999 over all compared outputs, max |dO| <= 5e-2 on rows
+that see at least 64 keys, and on every row the bound that e4m3 rounding of P
+and V (relative 2^-4 each) allows, 2^-3 * max|V|; |dLSE| <= 5e-2.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_134_b200 as attn
+import oracle
+from oracle import quant8 as oq8
+from synthetic import WORKLOADS, Workload, bf16_bits, make_qkv, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    attn.lib()
+
+
+def _regions(ws_host, off, B, Hq, Hkv, Nq, Nkv, d):
+    nqb, nkb = -(-Nq // 128), -(-Nkv // 128)
+
+    def r(i, dtype, shape):
+        n = int(np.prod(shape)) * np.dtype(dtype).itemsize
+        return ws_host[off[i]:off[i] + n].view(dtype).reshape(shape)
+    return {
+        "q8": r(0, np.int8, (B, Hq, Nq, d)), "k8": r(1, np.int8, (B, Hkv, Nkv, d)),
+        "v8": r(2, np.uint8, (B, Hkv, Nkv, d)), "sq": r(3, np.float32, (B, Hq, nqb)),
+        "sk": r(4, np.float32, (B, Hkv, nkb)), "sv": r(5, np.float32, (B, Hkv, d)),
+        "kbar": r(6, np.float32, (B, Hkv, d)), "qk": r(7, np.float32, (B, Hq, Nq)),
+    }
+
+
+def _check_prepass(B, Hq, Hkv, Nq, Nkv, d, seed, dist="normal"):
+    q, k, v = make_qkv(B, Hq, Hkv, Nq, Nkv, d, seed, dist)
+    ws = torch.empty(attn.q8_workspace_size(B, Hq, Hkv, Nq, Nkv, d), dtype=torch.uint8, device="cuda")
+    attn.q8_prepass(q.cuda(), k.cuda(), v.cuda(), ws)
+    st, where = attn.get_status()
+    assert st == 0, (st, where)
+    g = _regions(ws.cpu().numpy(), attn.q8_workspace_offsets(B, Hq, Hkv, Nq, Nkv, d), B, Hq, Hkv, Nq, Nkv, d)
+    qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
+    kbar = oq8.k_channel_mean(kb)
+    k8, sk = oq8.quant_int8_blocks(oq8.smooth_k(kb, kbar))
+    q8, sq = oq8.quant_int8_blocks(oracle.widen_bf16(qb).astype(np.float32))
+    v8, sv = oq8.quant_v_fp8(vb)
+    qk = oq8.q_dot_kbar(qb, kbar, Hkv)
+    assert np.array_equal(g["kbar"].view(np.uint32), kbar.view(np.uint32))
+    assert np.array_equal(g["sv"].view(np.uint32), sv.view(np.uint32))
+    assert np.array_equal(g["sq"].view(np.uint32), sq.view(np.uint32))
+    assert np.array_equal(g["sk"].view(np.uint32), sk.view(np.uint32))
+    assert np.array_equal(g["q8"], q8)
+    assert np.array_equal(g["k8"], k8)
+    assert np.array_equal(g["v8"], v8)
+    assert np.max(np.abs(g["qk"] - qk) / (1.0 + np.abs(qk))) < 1e-5
+
+
+@pytest.mark.parametrize("shape", [
+    (1, 2, 2, 256, 256, 128), (1, 4, 2, 300, 300, 128), (2, 4, 4, 513, 77, 64), (1, 2, 1, 1, 1, 128),
+])
+def test_prepass_bit_exact_small(shape):
+    _check_prepass(*shape, seed=sum(shape), dist="outlier_k")
+
+
+def test_prepass_bit_exact_8k_outlier_workload():
+    w = WORKLOADS["q8_8k_outlier"]
+    _check_prepass(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.seed, w.dist)
+
+
+def _check_fwd(B, Hq, Hkv, Nq, Nkv, d, causal, seed, dist="normal", n_rows=None):
+    q, k, v = make_qkv(B, Hq, Hkv, Nq, Nkv, d, seed, dist)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = attn.attn_fwd_q8(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+    st, where = attn.get_status()
+    assert st == 0, (st, where)
+    rows = None
+    if n_rows:
+        rows = sample_rows(Workload("t", B, Hq, Hkv, Nq, Nkv, d, causal, seed), n_rows)
+    O, L = oracle.attention_fp64(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, scale, rows=rows)
+    og = o.cpu().float().numpy().astype(np.float64)
+    lg = lse.cpu().numpy().astype(np.float64)
+    idx = np.arange(Nq)[None, None, :].repeat(B, 0).repeat(Hq, 1) if rows is None else rows
+    og = np.take_along_axis(og, idx[..., None], axis=2)
+    lg = np.take_along_axis(lg, idx, axis=2)
+    assert np.all(np.isfinite(og)) and np.all(np.isfinite(lg))
+    cos = float((og * O).sum() / math.sqrt((og * og).sum() * (O * O).sum()))
+    err = np.abs(og - O)
+    nkeys = (idx + 1) if causal else np.full_like(idx, Nkv)
+    many = nkeys >= 64
+    vmax = float(np.abs(oracle.widen_bf16(bf16_bits(v))).max())
+    assert cos >= 0.999, cos
+    if many.any():
+        assert err[many].max() <= 5e-2, err[many].max()
+    assert err.max() <= 2.0 ** -3 * vmax, (err.max(), vmax)
+    assert np.abs(lg - L).max() <= 5e-2
+    return cos, err.max()
+
+
+@pytest.mark.parametrize("shape", [
+    (1, 2, 2, 256, 256, 128, True), (1, 4, 2, 300, 300, 128, False), (2, 4, 4, 513, 513, 64, True),
+    (1, 2, 1, 100, 333, 128, False), (1, 8, 2, 1024, 1024, 128, True), (1, 2, 2, 1, 1, 64, True),
+])
+def test_q8_forward_small(shape):
+    _check_fwd(*shape, seed=sum(shape) + 3, dist="outlier_k")
+
+
+@pytest.mark.parametrize("name", ["q8_8k_outlier", "q8_8k_normal"])
+def test_q8_forward_workloads(name):
+    w = WORKLOADS[name]
+    _check_fwd(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.causal, w.seed, w.dist, n_rows=w.oracle_rows)
+
+
+def test_q8_workspace_errors():
+    q, k, v = make_qkv(1, 2, 2, 128, 128, 128, seed=1)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    need = attn.q8_workspace_size(1, 2, 2, 128, 128, 128)
+    small = torch.empty(need - 1, dtype=torch.uint8, device="cuda")
+    with pytest.raises(attn.AttnError) as e:
+        attn.attn_fwd_q8(q, k, v, workspace=small)
+    assert e.value.status == 6
