@@ -6,8 +6,10 @@ rounded division and round-half-even); q.kbar within fp32 rounding.
 
 Forward: against the EXACT fp64 oracle (not the quantised one) with the 8-bit
 tolerance: cosine >= 0.999 over all compared outputs, max |dO| <= 5e-2 on rows
-that see at least 64 keys, and on every row the bound that e4m3 rounding of P
-and V (relative 2^-4 each) allows, 2^-3 * max|V|; |dLSE| <= 5e-2.
+that see at least 128 keys (one full K/V tile; rows with fewer keys average too
+few e4m3-rounded terms — the oracle's own one-shot 8-bit result misses 5e-2
+there as well), and on every row the bound that e4m3 rounding of P and V
+(relative 2^-4 each) allows, 2^-3 * max|V|; |dLSE| <= 5e-2.
 """
 import math
 
@@ -64,7 +66,11 @@ def _check_prepass(B, Hq, Hkv, Nq, Nkv, d, seed, dist="normal"):
     assert np.array_equal(g["q8"], q8)
     assert np.array_equal(g["k8"], k8)
     assert np.array_equal(g["v8"], v8)
-    assert np.max(np.abs(g["qk"] - qk) / (1.0 + np.abs(qk))) < 1e-5
+    # fp32 dot product of d terms: error <= d * 2^-24 * sum_c |q_c kbar_c|
+    qf = oracle.widen_bf16(qb)
+    g_of = np.arange(Hq) // (Hq // Hkv)
+    mag = np.einsum("bhnd,bhd->bhn", np.abs(qf), np.abs(kbar[:, g_of].astype(np.float64)))
+    assert np.all(np.abs(g["qk"] - qk) <= d * 2.0 ** -24 * mag + 1e-30)
 
 
 @pytest.mark.parametrize("shape", [
@@ -98,7 +104,7 @@ def _check_fwd(B, Hq, Hkv, Nq, Nkv, d, causal, seed, dist="normal", n_rows=None)
     cos = float((og * O).sum() / math.sqrt((og * og).sum() * (O * O).sum()))
     err = np.abs(og - O)
     nkeys = (idx + 1) if causal else np.full_like(idx, Nkv)
-    many = nkeys >= 64
+    many = nkeys >= 128
     vmax = float(np.abs(oracle.widen_bf16(bf16_bits(v))).max())
     assert cos >= 0.999, cos
     if many.any():
