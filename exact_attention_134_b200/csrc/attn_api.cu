@@ -217,6 +217,30 @@ HostLayout host_layout(int B, int Hq, int Hkv, int Nq, int Nkv, int d) {
 
 }  // namespace
 
+namespace attn_sm100 {
+
+// Internal: the argument checks of attn_fwd / attn_fwd_q8.
+attn_status_t validate_fwd_args(const void* q, const void* k, const void* v, const void* o,
+                                const void* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                                int causal, float scale) {
+  return check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+}
+
+// Internal: validate arguments and run the 8-bit forward with a workspace the
+// caller already has (used by the entry point whose workspace is a static
+// device array).
+attn_status_t q8_forward_with_workspace(const void* q, const void* k, const void* v, void* o,
+                                        float* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                                        int causal, float scale, void* workspace,
+                                        size_t workspace_bytes, cudaStream_t stream) {
+  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  if (s != ATTN_OK) return s;
+  return run_q8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, workspace, workspace_bytes,
+                false, stream);
+}
+
+}  // namespace attn_sm100
+
 extern "C" {
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,

@@ -57,6 +57,15 @@ struct Q8Launch {
 
 cudaError_t launch_q8(const Q8Launch& L, int d, cudaStream_t stream);
 
+attn_status_t validate_fwd_args(const void* q, const void* k, const void* v, const void* o,
+                                const void* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                                int causal, float scale);
+
+attn_status_t q8_forward_with_workspace(const void* q, const void* k, const void* v, void* o,
+                                        float* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                                        int causal, float scale, void* workspace,
+                                        size_t workspace_bytes, cudaStream_t stream);
+
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& to, const FwdParams& p, int B, int Hq, int d,
                             cudaStream_t stream);

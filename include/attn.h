@@ -112,6 +112,35 @@ ATTN_API attn_status_t attn_fwd_q8(const void* q, const void* k, const void* v, 
                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_fwd_q8_noalloc — attn_fwd_q8 for callers that cannot allocate device
+ * memory, e.g. a plugin inside another framework's inference engine that is
+ * handed only its input and output buffers, or a program that must not call
+ * cudaMalloc while serving (it can synchronise the device, and fails when
+ * another allocator has reserved the GPU's memory). The pages have no
+ * counterpart: this is an interface convenience, not part of the method.
+ *   arguments      as attn_fwd (bf16 q, k, v; bf16 o; fp32 lse); no workspace
+ *   scratch        a static device array of attn_fwd_q8_static_scratch_bytes()
+ *                  bytes (32 MiB) inside the library, held on every GPU that
+ *                  loads the library until the process exits
+ *   size limit     problems whose attn_fwd_q8_workspace_size() exceeds the
+ *                  array are rejected with ATTN_ERR_WORKSPACE before anything
+ *                  is queued
+ *   allocation     none: no cudaMalloc / cudaFree or allocating library call
+ *   first call     on each device, looks up the array's device address
+ *                  (cudaGetSymbolAddress) with that device current; make the
+ *                  first call on a device before any stream capture
+ *   concurrency    every call shares the one array: calls whose work overlaps
+ *                  on the GPU (different streams, no ordering between them)
+ *                  race on it and must be serialised by the caller. The array
+ *                  keeps the last call's contents; nothing in it needs to
+ *                  start at zero.
+ */
+ATTN_API size_t attn_fwd_q8_static_scratch_bytes(void);
+ATTN_API attn_status_t attn_fwd_q8_noalloc(const void* q, const void* k, const void* v, void* o,
+                                           float* lse, int B, int Hq, int Hkv, int Nq, int Nkv,
+                                           int d, int causal, float scale, void* stream);
+
+/*
  * attn_q8_prepass — only the three prepass launches of attn_fwd_q8 (K mean,
  * V channel scales, quantisation of Q, K, V), writing the workspace; used to
  * time the prepass on its own and to inspect its results.
