@@ -151,13 +151,20 @@ def _barrier(world):
 
 
 def _max_over_ranks(x: float, world: int) -> float:
+    """Timing only (not on the data path): the slowest rank's time."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    on_gpu = dist.get_backend() == "nccl"
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if on_gpu else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_tflops(flops_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job throughput: all ranks' work over the slowest rank's time."""
+    return world * flops_per_rank / (max_ms * 1e-3) / 1e12
 
 
 def rank_workload(w: Workload, rank: int) -> Workload:
@@ -321,7 +328,7 @@ def run_ours(args):
     res = bench_workload(w, args.steps, args.warmup, world, rank, attn)
     clk = clocks.stop()
     ms = res["total_ms"] / args.steps
-    value = world * w.flops / (ms * 1e-3) / 1e12
+    value = aggregate_tflops(w.flops, world, ms)
     per_launch_tflops = w.flops / (statistics.mean(res["times"]) * 1e-3) / 1e12
     e2e = None
     if not args.kernel_only:
