@@ -51,6 +51,9 @@ struct FwdCfg {
   static constexpr int kTileBytes = kBM * D * 2;
   static constexpr int kBoxes = D / 64;
   static constexpr int kStages = (D == 128) ? 4 : 8;
+  // of every 4 pairs of exponentials, this many are evaluated by the FMA-pipe
+  // polynomial instead of MUFU (MUFU is the co-bottleneck with the tensor pipe)
+  static constexpr int kEmuPairs = (D == 128) ? 1 : 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffRing = 2 * kTileBytes;
   static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
@@ -108,7 +111,7 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(200)
     attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v,
@@ -329,40 +332,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
       tmem_wait_ld();
 
-      // mask: keys >= Nkv, and (causal) keys after this row
+      // mask keys >= Nkv and (causal) keys after the row, only on tiles that need it
       const int kv0 = j * kBN;
-      int lim = p.Nkv - kv0;
-      if (p.causal) lim = min(lim, row - kv0 + 1);
-      if (lim < kBN) {
+      const bool tile_masked =
+          (kv0 + kBN > p.Nkv) || (p.causal && kv0 + kBN - 1 > q0 + t * kBM);
+      if (tile_masked) {
+        int lim = p.Nkv - kv0;
+        if (p.causal) lim = min(lim, row - kv0 + 1);
 #pragma unroll
         for (int c = 0; c < kBN; ++c)
           if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
       }
-      float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
-      float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int c = 4; c < kBN; c += 4) {
-        mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
-        mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
-        mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
-        mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
+      for (int c = 0; c < kBN; c += 8) {
+        mx0 = fmax3(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+        mx1 = fmax3(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+        mx2 = fmax3(mx2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+        mx3 = fmax3(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
       }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float m_tile = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
       float alpha = 1.0f;
       if (m_tile > m_run + kRescaleThreshold) {
         alpha = ex2_approx(m_run - m_tile);  // 0 on the first visible tile
         m_run = m_tile;
       }
       const float mb = (m_run == -INFINITY) ? 0.0f : m_run;
-      float sum0 = 0.f, sum1 = 0.f;
+      const float2 slope = make_float2(sl2, sl2), bias = make_float2(-mb, -mb);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
+      // p = 2^(s * scale * log2(e) - m); P packed to bf16 in place (index pi <= 2 pi)
+      if (tile_masked) {
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -mb));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), sl2, -mb));
-        sum0 += p0;
-        sum1 += p1;
-        sr[c >> 1] = pack_bf16x2(p0, p1);  // P packed in place (index c/2 <= c already read)
+        for (int pi = 0; pi < kBN / 2; ++pi) {
+          const float2 x = fma2(make_float2(__uint_as_float(sr[2 * pi]), __uint_as_float(sr[2 * pi + 1])),
+                                slope, bias);
+          const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          acc[pi & 3] = add2(acc[pi & 3], e);
+          sr[pi] = pack_bf16x2(e.x, e.y);
+        }
+      } else {
+        // a fixed share of the exponentials runs on the FMA pipe, the rest on MUFU
+#pragma unroll
+        for (int pi = 0; pi < kBN / 2; ++pi) {
+          const float2 x = fma2(make_float2(__uint_as_float(sr[2 * pi]), __uint_as_float(sr[2 * pi + 1])),
+                                slope, bias);
+          const float2 e = ((pi & 3) < C::kEmuPairs) ? exp2_poly2(x)
+                                                     : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          acc[pi & 3] = add2(acc[pi & 3], e);
+          sr[pi] = pack_bf16x2(e.x, e.y);
+        }
       }
+      const float2 acc01 = add2(acc[0], acc[1]), acc23 = add2(acc[2], acc[3]);
+      const float row_sum = (acc01.x + acc01.y) + (acc23.x + acc23.y);
       tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&sr[0]));
       tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&sr[32]));
 
@@ -379,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(tO + 32 * c, o);
         }
       }
-      l_run = l_run * alpha + (sum0 + sum1);
+      l_run = l_run * alpha + row_sum;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(BarLayout::kPFull + t));

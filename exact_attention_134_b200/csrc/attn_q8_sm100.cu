@@ -293,7 +293,7 @@ __device__ __forceinline__ void issue_pv_f8(uint32_t o_tmem, uint32_t p_tmem, ui
 }
 
 template <int D>
-__global__ void __launch_bounds__(kQ8Threads, 1)
+__global__ void __maxnreg__(200)
     attn_fwd_q8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                        const Q8Params p) {
@@ -501,43 +501,67 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
         tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
       tmem_wait_ld();
       const float f = sq_t * p.sk[(size_t)bh_kv * p.nkb + j] * p.scale_log2;
-      const int kv0 = j * kTok;
-      int lim = p.Nkv - kv0;
-      if (p.causal) lim = min(lim, row - kv0 + 1);
+      // s32 -> fp32 without the conversion unit: |s| <= 127 * 127 * d < 2^22, so
+      // the bits of (s + 0x4B400000) are the float 1.5 * 2^23 + s exactly
+      constexpr float kMagic = 12582912.0f;
 #pragma unroll
-      for (int c = 0; c < kTok; ++c) {
-        const float sf = static_cast<float>(static_cast<int>(sr[c]));
-        sr[c] = __float_as_uint(c < lim ? sf : -INFINITY);
+      for (int c = 0; c < kTok; c += 2) {
+        const float2 v = add2(make_float2(__uint_as_float(sr[c] + 0x4B400000u),
+                                          __uint_as_float(sr[c + 1] + 0x4B400000u)),
+                              make_float2(-kMagic, -kMagic));
+        sr[c] = __float_as_uint(v.x);
+        sr[c + 1] = __float_as_uint(v.y);
       }
-      float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
-      float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
+      const int kv0 = j * kTok;
+      const bool tile_masked =
+          (kv0 + kTok > p.Nkv) || (p.causal && kv0 + kTok - 1 > q0 + t * kTok);
+      if (tile_masked) {
+        int lim = p.Nkv - kv0;
+        if (p.causal) lim = min(lim, row - kv0 + 1);
 #pragma unroll
-      for (int c = 4; c < kTok; c += 4) {
-        mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
-        mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
-        mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
-        mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
+        for (int c = 0; c < kTok; ++c)
+          if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kTok; c += 8) {
+        mx0 = fmax3(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+        mx1 = fmax3(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+        mx2 = fmax3(mx2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+        mx3 = fmax3(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
       }
       // f > 0 (all scales positive), so the max of s*f is f * max(s)
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * f;
+      const float m_tile = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * f;
       float alpha = 1.0f;
       if (m_tile > m_run) {
         alpha = ex2_approx(m_run - m_tile);
         m_run = m_tile;
       }
       const float mb = (m_run == -INFINITY) ? 0.0f : m_run;
-      const float bias = kLog2_448 - mb;  // p448 = 448 * 2^(s*f - m) = 2^(s*f - m + log2 448)
-      float sum0 = 0.f, sum1 = 0.f;
+      // p448 = 448 * 2^(s*f - m) = 2^(s*f - m + log2 448)
+      const float2 slope = make_float2(f, f), bias = make_float2(kLog2_448 - mb, kLog2_448 - mb);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < kTok; c += 4) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c]), f, bias));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), f, bias));
-        const float p2 = ex2_approx(fmaf(__uint_as_float(sr[c + 2]), f, bias));
-        const float p3 = ex2_approx(fmaf(__uint_as_float(sr[c + 3]), f, bias));
-        sum0 += p0 + p2;
-        sum1 += p1 + p3;
-        sr[c >> 2] = pack_e4m3x2(p0, p1) | (pack_e4m3x2(p2, p3) << 16);
+      for (int qd = 0; qd < kTok / 4; ++qd) {
+        const float2 x0 = fma2(make_float2(__uint_as_float(sr[4 * qd]), __uint_as_float(sr[4 * qd + 1])),
+                               slope, bias);
+        const float2 x1 = fma2(make_float2(__uint_as_float(sr[4 * qd + 2]), __uint_as_float(sr[4 * qd + 3])),
+                               slope, bias);
+        float2 e0, e1;
+        if (!tile_masked && (qd & 1)) {
+          // half of the exponentials of unmasked tiles run on the FMA pipe
+          e0 = exp2_poly2(x0);
+          e1 = exp2_poly2(x1);
+        } else {
+          e0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+          e1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+        }
+        acc[qd & 3] = add2(acc[qd & 3], add2(e0, e1));
+        sr[qd] = pack_e4m3x2(e0.x, e0.y) | (pack_e4m3x2(e1.x, e1.y) << 16);
       }
+      const float2 acc01 = add2(acc[0], acc[1]), acc23 = add2(acc[2], acc[3]);
+      const float row_sum = (acc01.x + acc01.y) + (acc23.x + acc23.y);
       tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&sr[0]));
       const bool rescale = (j > 0) && (alpha != 1.0f);
       if (__any_sync(0xffffffffu, rescale)) {
@@ -551,7 +575,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
           tmem_st32(tO + 32 * c, o);
         }
       }
-      l_run = l_run * alpha + (sum0 + sum1);
+      l_run = l_run * alpha + row_sum;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(Q8Bar::kPFull + t));

@@ -298,6 +298,63 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// ---------------------------------------------------------------- packed fp32 (sm_100)
+__device__ __forceinline__ uint64_t f2_bits(float2 a) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a.x), "f"(a.y));
+  return r;
+}
+
+__device__ __forceinline__ float2 bits_f2(uint64_t r) {
+  float2 a;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a.x), "=f"(a.y) : "l"(r));
+  return a;
+}
+
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return bits_f2(r);
+}
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(r);
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x on the FMA pipe for a pair of arguments x <= 127. Cody–Waite range
+// reduction (Cody & Waite, "Software Manual for the Elementary Functions",
+// 1980): j = round(x) via the 1.5 * 2^23 addition trick, f = x - j in
+// [-1/2, 1/2], 2^f from a degree-3 polynomial whose coefficients minimise the
+// maximum relative error on that interval (Remez exchange; fitted by
+// csrc/exp2_poly_fit.py; max relative error 7.5e-5), then j is added to the
+// exponent field. Arguments below -125 are clamped (result ~2^-125 instead of
+// a smaller number; the clamp also keeps the exponent field of the result
+// normal), so only call it where that is harmless: for softmax weights below
+// 2^-125 of the row maximum's.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = add2(x, make_float2(kRound, kRound));
+  const float2 j = add2(t, make_float2(-kRound, -kRound));
+  const float2 f = fma2(j, make_float2(-1.0f, -1.0f), x);
+  const float c0 = __uint_as_float(0x3f7ffb49u), c1 = __uint_as_float(0x3f31798du);
+  const float c2 = __uint_as_float(0x3e786f0du), c3 = __uint_as_float(0x3d61fbb0u);
+  float2 p = fma2(f, make_float2(c3, c3), make_float2(c2, c2));
+  p = fma2(p, f, make_float2(c1, c1));
+  p = fma2(p, f, make_float2(c0, c0));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in bits 0..15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
