@@ -53,6 +53,7 @@ _SIGNATURES = {
     "attn_set_timeout_ms": (_c_int, [_c_int]),
     "attn_status_string": (ctypes.c_char_p, [_c_int]),
     "attn_version": (_c_int, []),
+    "attn_last_cuda_error": (_c_int, [ctypes.POINTER(ctypes.c_char_p)]),
 }
 
 
@@ -76,6 +77,10 @@ def lib() -> ctypes.CDLL:
 
 def _check(status: int, what: str):
     if status != 0:
+        if status == 4:
+            msg = ctypes.c_char_p()
+            code = lib().attn_last_cuda_error(ctypes.byref(msg))
+            what = f"{what} (cuda error {code}: {msg.value.decode() if msg.value else ''})"
         raise AttnError(status, what)
 
 

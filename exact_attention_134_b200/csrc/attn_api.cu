@@ -22,6 +22,15 @@ std::once_flag g_encode_once;
 std::mutex g_dev_mutex;
 int* g_status_ptr[kMaxDevices] = {nullptr};
 std::atomic<long long> g_timeout_ns{1000000000LL};
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+// Map a CUDA runtime result to the ABI status, remembering the runtime's code
+// for attn_last_cuda_error().
+attn_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return ATTN_OK;
+  g_last_cuda_error = e;
+  return ATTN_ERR_CUDA;
+}
 
 void load_encode() {
   void* fn = nullptr;
@@ -118,8 +127,7 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.num_row_blocks = (Nq + rows - 1) / rows;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
-  cudaError_t e = attn_sm100::launch_fwd_bf16(tq, tk, tv, to, p, B, Hq, d, stream);
-  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return cuda_status(attn_sm100::launch_fwd_bf16(tq, tk, tv, to, p, B, Hq, d, stream));
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -194,8 +202,7 @@ attn_status_t run_q8(const void* q, const void* k, const void* v, void* o, float
         !make_map(&L.to, o, d, Nq, (long long)B * Hq))
       return ATTN_ERR_CUDA;
   }
-  cudaError_t e = attn_sm100::launch_q8(L, d, stream);
-  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return cuda_status(attn_sm100::launch_q8(L, d, stream));
 }
 
 struct HostLayout {
@@ -355,5 +362,10 @@ const char* attn_status_string(attn_status_t s) {
 }
 
 int attn_version(void) { return 100; }
+
+int attn_last_cuda_error(const char** message) {
+  if (message) *message = cudaGetErrorString(g_last_cuda_error);
+  return static_cast<int>(g_last_cuda_error);
+}
 
 }  // extern "C"

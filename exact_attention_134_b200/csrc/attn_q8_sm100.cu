@@ -293,7 +293,7 @@ __device__ __forceinline__ void issue_pv_f8(uint32_t o_tmem, uint32_t p_tmem, ui
 }
 
 template <int D>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kQ8Threads, 1)
     attn_fwd_q8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                        const Q8Params p) {

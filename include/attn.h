@@ -180,6 +180,11 @@ ATTN_API attn_status_t attn_set_timeout_ms(int ms);
 /* Human-readable name of a status code (static storage). */
 ATTN_API const char* attn_status_string(attn_status_t status);
 
+/* attn_last_cuda_error — the CUDA runtime error code behind the most recent
+ * ATTN_ERR_CUDA returned on this host thread by a launch (0 if none), and
+ * its message in *message (static storage) when message is not NULL. */
+ATTN_API int attn_last_cuda_error(const char** message);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 ATTN_API int attn_version(void);
 
