@@ -21,6 +21,7 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 std::mutex g_dev_mutex;
 int* g_status_ptr[kMaxDevices] = {nullptr};
+int g_sm_count[kMaxDevices] = {0};
 std::atomic<long long> g_timeout_ns{1000000000LL};
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
@@ -52,9 +53,20 @@ int* device_status_ptr() {
   if (!g_status_ptr[dev]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) return nullptr;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      return nullptr;
+    g_sm_count[dev] = sms;
     g_status_ptr[dev] = static_cast<int*>(ptr);
   }
   return g_status_ptr[dev];
+}
+
+// SM count of the current device (valid after device_status_ptr() succeeded).
+int device_sm_count() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return g_sm_count[dev];
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -118,6 +130,7 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   attn_sm100::FwdParams p;
   p.lse = lse;
   p.status = status;
+  p.B = B;
   p.Nq = Nq;
   p.Nkv = Nkv;
   p.Hq = Hq;
@@ -125,9 +138,13 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.causal = causal;
   const int rows = attn_sm100::fwd_rows_per_cta();
   p.num_row_blocks = (Nq + rows - 1) / rows;
+  const long long units = (long long)B * Hq * p.num_row_blocks;
+  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  p.num_units = (int)units;
+  p.num_ctas = device_sm_count();
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
-  return cuda_status(attn_sm100::launch_fwd_bf16(tq, tk, tv, to, p, B, Hq, d, stream));
+  return cuda_status(attn_sm100::launch_fwd_bf16(tq, tk, tv, to, p, d, stream));
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

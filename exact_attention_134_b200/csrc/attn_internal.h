@@ -14,9 +14,11 @@ namespace attn_sm100 {
 struct FwdParams {
   float* lse;                     // fp32 [B, Hq, Nq]
   int* status;                    // device status word: [0] code, [1] where
-  int Nq, Nkv, Hq, Hkv;
+  int B, Nq, Nkv, Hq, Hkv;
   int causal;
-  int num_row_blocks;             // ceil(Nq / rows per CTA)
+  int num_row_blocks;             // ceil(Nq / rows per work unit)
+  int num_units;                  // B * Hq * num_row_blocks
+  int num_ctas;                   // persistent grid size (SM count)
   float scale_log2;               // scale * log2(e)
   unsigned long long timeout_ns;  // budget of every pipeline wait
 };
@@ -67,8 +69,7 @@ attn_status_t q8_forward_with_workspace(const void* q, const void* k, const void
                                         size_t workspace_bytes, cudaStream_t stream);
 
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& to, const FwdParams& p, int B, int Hq, int d,
-                            cudaStream_t stream);
+                            const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t stream);
 int fwd_rows_per_cta();
 
 }  // namespace attn_sm100

@@ -241,6 +241,23 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+// ---------------------------------------------------------------- registers
+// Re-split the register file between warpgroups (all four warps of a
+// warpgroup execute it). The per-sub-partition sum of the new limits must not
+// exceed what the CTA was launched with.
+template <int N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ void tma_store_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor (tcgen05 format, version 1) for a tile laid
 // out in the 128-byte swizzle pattern the TMA unit writes (8-row x 128-byte
