@@ -128,6 +128,7 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
       !make_map(&tv, v, d, Nkv, (long long)B * Hkv) || !make_map(&to, o, d, Nq, (long long)B * Hq))
     return ATTN_ERR_CUDA;
   attn_sm100::FwdParams p;
+  p.o = o;
   p.lse = lse;
   p.status = status;
   p.B = B;
@@ -141,7 +142,11 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   const long long units = (long long)B * Hq * p.num_row_blocks;
   if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   p.num_units = (int)units;
+#ifdef ATTN_ONE_UNIT_PER_CTA
+  p.num_ctas = p.num_units;
+#else
   p.num_ctas = device_sm_count();
+#endif
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
   return cuda_status(attn_sm100::launch_fwd_bf16(tq, tk, tv, to, p, d, stream));

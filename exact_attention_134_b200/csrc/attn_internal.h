@@ -12,6 +12,7 @@ namespace attn_sm100 {
 
 // Kernel parameters of the bf16 forward (tensor maps are passed separately).
 struct FwdParams {
+  void* o;                        // bf16 [B, Hq, Nq, d]
   float* lse;                     // fp32 [B, Hq, Nq]
   int* status;                    // device status word: [0] code, [1] where
   int B, Nq, Nkv, Hq, Hkv;
