@@ -210,8 +210,15 @@ def bench_workload(w: Workload, steps: int, warmup: int, world: int, rank: int, 
         flush = lambda: scratch.zero_()  # noqa: E731
         l2_mode = "l2_flushed_between_steps"
 
-    def step():
-        lib_mod.attn_fwd(qd, kd, vd, causal=w.causal, out=o, lse=lse)
+    if w.path == "q8":
+        ws = torch.empty(lib_mod.q8_workspace_size(wr.B, wr.Hq, wr.Hkv, wr.Nq, wr.Nkv, wr.d),
+                         dtype=torch.uint8, device="cuda")
+
+        def step():
+            lib_mod.attn_fwd_q8(qd, kd, vd, causal=w.causal, workspace=ws, out=o, lse=lse)
+    else:
+        def step():
+            lib_mod.attn_fwd(qd, kd, vd, causal=w.causal, out=o, lse=lse)
 
     for _ in range(max(warmup, 3)):
         step()
@@ -331,7 +338,7 @@ def run_ours(args):
     value = aggregate_tflops(w.flops, world, ms)
     per_launch_tflops = w.flops / (statistics.mean(res["times"]) * 1e-3) / 1e12
     e2e = None
-    if not args.kernel_only:
+    if not args.kernel_only and w.path != "q8":
         e2e_steps = max(2, args.steps // 2)
         e2e_ms, h2d, d2h = bench_e2e(w, e2e_steps, 1, world, rank, attn)
         e2e = {"value": round(world * w.flops / (e2e_ms / e2e_steps * 1e-3) / 1e12, 2),
@@ -379,18 +386,20 @@ def run_ours(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16",
+            "dtype": "bf16" if w.path != "q8" else "int8 QK^T + e4m3 PV (fp32 accumulation)",
             "data": "synthetic (seeded torch CPU randn -> bf16; outlier-K offsets per head/channel)",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq,
                        "Nkv": w.Nkv, "d": w.d, "causal": w.causal, "scale": "1/sqrt(d)",
                        "l2": res["l2"], "per_rank": "independent batch (seed + 1000*rank)"},
             "frac_of_bf16_peak": round(value / world / peaks["bf16"], 4),
             "roofline": {"bound": "tensor", "achieved": round(per_launch_tflops, 2),
-                         "peak": peaks["bf16"], "unit": "TFLOP/s",
-                         "frac": round(per_launch_tflops / peaks["bf16"], 4),
+                         "peak": peaks["bf16"] * (2 if w.path == "q8" else 1), "unit": "TFLOP/s",
+                         "frac": round(per_launch_tflops / (peaks["bf16"] * (2 if w.path == "q8" else 1)), 4),
                          "traffic": traffic,
-                         "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
-                         "kernel": "attn_fwd_bf16_kernel",
+                         "peak_source": (f"{peaks['source']} bf16 burst (cuBLAS)" if w.path != "q8" else
+                                         f"2 x {peaks['source']} bf16 burst (nominal fp8/bf16 ratio)"),
+                         "kernel": "attn_fwd_bf16_kernel" if w.path != "q8" else
+                                   "attn_fwd_q8 (3 prepass kernels + main kernel)",
                          "algorithmic_min_bytes": w.min_hbm_bytes},
             "e2e": e2e,
             "gpu_launches": args.steps,

@@ -32,6 +32,11 @@ namespace attn_sm100 {
 namespace {
 
 constexpr int kQ8Threads = 320;
+#ifndef ATTN_Q8_EMU
+#define ATTN_Q8_EMU 0
+#endif
+// 1: half of the exponentials of unmasked tiles use the FMA-pipe polynomial
+constexpr bool kQ8EmuHalf = ATTN_Q8_EMU != 0;
 constexpr int kTok = 128;         // tokens per quantisation block == MMA tile rows
 constexpr int kPrepThreads = 256;
 
@@ -549,7 +554,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
         const float2 x1 = fma2(make_float2(__uint_as_float(sr[4 * qd + 2]), __uint_as_float(sr[4 * qd + 3])),
                                slope, bias);
         float2 e0, e1;
-        if (!tile_masked && (qd & 1)) {
+        if (kQ8EmuHalf && !tile_masked && (qd & 1)) {
           // half of the exponentials of unmasked tiles run on the FMA pipe
           e0 = exp2_poly2(x0);
           e1 = exp2_poly2(x1);
