@@ -50,8 +50,20 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
   f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
 }
 
-__device__ __forceinline__ int8_t quant_i8(float x, float s) {
-  int c = __float2int_rn(__fdiv_rn(x, s));  // round half to even
+// x / s rounded to nearest, without a division per element: with r = RN(1/s)
+// (computed once per scale), q0 = RN(x * r) is within an ulp of x / s, the
+// residual x - q0 * s is exact in one FMA, and RN(q0 + residual * r) is the
+// correctly rounded quotient for normal operands (Markstein's FMA correction,
+// P. Markstein, IBM J. Res. Dev. 34(1), 1990). The prepass tests compare the
+// resulting codes bit for bit with division on the host.
+__device__ __forceinline__ float div_rn(float x, float s, float r) {
+  const float q0 = x * r;
+  const float e = fmaf(-q0, s, x);
+  return fmaf(e, r, q0);
+}
+
+__device__ __forceinline__ int8_t quant_i8(float x, float s, float r) {
+  int c = __float2int_rn(div_rn(x, s, r));  // round half to even
   c = c > 127 ? 127 : (c < -127 ? -127 : c);
   return static_cast<int8_t>(c);
 }
@@ -86,13 +98,20 @@ __global__ void __launch_bounds__(kPrepThreads)
   float mx[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) { s[i] = 0.0; mx[i] = 0.0f; }
-  for (int r = rs; r < kTok; r += RPP) {
-    const int t = t0 + r;
-    if (t >= Nkv) break;
-    const size_t off = (bh * Nkv + t) * D + vc * 8;
+  constexpr int NP = kTok / RPP;
+  uint4 kv[NP], vv[NP];
+#pragma unroll
+  for (int pp = 0; pp < NP; ++pp) {  // issue every load of the chunk before using any
+    const int t = t0 + rs + pp * RPP;
+    const size_t off = (bh * Nkv + (t < Nkv ? t : 0)) * D + vc * 8;
+    kv[pp] = t < Nkv ? *reinterpret_cast<const uint4*>(k + off) : make_uint4(0, 0, 0, 0);
+    vv[pp] = t < Nkv ? *reinterpret_cast<const uint4*>(v + off) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int pp = 0; pp < NP; ++pp) {
     float kf[8], vf[8];
-    unpack8(*reinterpret_cast<const uint4*>(k + off), kf);
-    unpack8(*reinterpret_cast<const uint4*>(v + off), vf);
+    unpack8(kv[pp], kf);
+    unpack8(vv[pp], vf);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       s[i] += static_cast<double>(kf[i]);
@@ -171,6 +190,7 @@ __global__ void __launch_bounds__(kPrepThreads)
     }
     amax = block_max256(amax, red);
     const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 1.0f;
+    const float rs = __frcp_rn(s);
     float kb[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) kb[i] = kbar[bhk * D + vc * 8 + i];
@@ -186,8 +206,8 @@ __global__ void __launch_bounds__(kPrepThreads)
         uint32_t lo = 0, hi = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          lo |= (uint32_t)(uint8_t)quant_i8(x[pp][i], s) << (8 * i);
-          hi |= (uint32_t)(uint8_t)quant_i8(x[pp][i + 4], s) << (8 * i);
+          lo |= (uint32_t)(uint8_t)quant_i8(x[pp][i], s, rs) << (8 * i);
+          hi |= (uint32_t)(uint8_t)quant_i8(x[pp][i + 4], s, rs) << (8 * i);
         }
         *reinterpret_cast<uint2*>(q8 + ((size_t)bh * Nq + t) * D + vc * 8) = make_uint2(lo, hi);
         if (vc == 0) qk[(size_t)bh * Nq + t] = dot;
@@ -198,11 +218,12 @@ __global__ void __launch_bounds__(kPrepThreads)
     tile -= n_q_tiles;
     const int kb_i = (int)(tile % nkb);
     const size_t bh = (size_t)(tile / nkb);  // b * Hkv + h
-    float kb[8], svc[8];
+    float kb[8], svc[8], rsv[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       kb[i] = kbar[bh * D + vc * 8 + i];
       svc[i] = sv[bh * D + vc * 8 + i];
+      rsv[i] = __frcp_rn(svc[i]);
     }
     float amax = 0.0f;
 #pragma unroll
@@ -221,6 +242,7 @@ __global__ void __launch_bounds__(kPrepThreads)
     }
     amax = block_max256(amax, red);
     const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 1.0f;
+    const float r_s = __frcp_rn(s);
 #pragma unroll
     for (int pp = 0; pp < NP; ++pp) {
       const int t = kb_i * kTok + rs + pp * RPP;
@@ -228,16 +250,17 @@ __global__ void __launch_bounds__(kPrepThreads)
         uint32_t lo = 0, hi = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          lo |= (uint32_t)(uint8_t)quant_i8(x[pp][i], s) << (8 * i);
-          hi |= (uint32_t)(uint8_t)quant_i8(x[pp][i + 4], s) << (8 * i);
+          lo |= (uint32_t)(uint8_t)quant_i8(x[pp][i], s, r_s) << (8 * i);
+          hi |= (uint32_t)(uint8_t)quant_i8(x[pp][i + 4], s, r_s) << (8 * i);
         }
         *reinterpret_cast<uint2*>(k8 + (bh * Nkv + t) * D + vc * 8) = make_uint2(lo, hi);
         float vf[8];
         unpack8(*reinterpret_cast<const uint4*>(v + (bh * Nkv + t) * D + vc * 8), vf);
-        uint32_t w0 = pack_e4m3x2(__fdiv_rn(vf[0], svc[0]), __fdiv_rn(vf[1], svc[1])) |
-                      (pack_e4m3x2(__fdiv_rn(vf[2], svc[2]), __fdiv_rn(vf[3], svc[3])) << 16);
-        uint32_t w1 = pack_e4m3x2(__fdiv_rn(vf[4], svc[4]), __fdiv_rn(vf[5], svc[5])) |
-                      (pack_e4m3x2(__fdiv_rn(vf[6], svc[6]), __fdiv_rn(vf[7], svc[7])) << 16);
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = div_rn(vf[i], svc[i], rsv[i]);
+        const uint32_t w0 = pack_e4m3x2(y[0], y[1]) | (pack_e4m3x2(y[2], y[3]) << 16);
+        const uint32_t w1 = pack_e4m3x2(y[4], y[5]) | (pack_e4m3x2(y[6], y[7]) << 16);
         *reinterpret_cast<uint2*>(v8 + (bh * Nkv + t) * D + vc * 8) = make_uint2(w0, w1);
       }
     }
