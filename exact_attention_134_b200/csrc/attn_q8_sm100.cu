@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kPrepThreads)
     }
     amax = block_max256(amax, red);
     const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 1.0f;
-    const float rs = __frcp_rn(s);
+    const float r_q = __frcp_rn(s);
     float kb[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) kb[i] = kbar[bhk * D + vc * 8 + i];
@@ -206,8 +206,8 @@ __global__ void __launch_bounds__(kPrepThreads)
         uint32_t lo = 0, hi = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          lo |= (uint32_t)(uint8_t)quant_i8(x[pp][i], s, rs) << (8 * i);
-          hi |= (uint32_t)(uint8_t)quant_i8(x[pp][i + 4], s, rs) << (8 * i);
+          lo |= (uint32_t)(uint8_t)quant_i8(x[pp][i], s, r_q) << (8 * i);
+          hi |= (uint32_t)(uint8_t)quant_i8(x[pp][i + 4], s, r_q) << (8 * i);
         }
         *reinterpret_cast<uint2*>(q8 + ((size_t)bh * Nq + t) * D + vc * 8) = make_uint2(lo, hi);
         if (vc == 0) qk[(size_t)bh * Nq + t] = dot;
