@@ -19,5 +19,6 @@ state (rows of P sum to 1, online softmax equals one-shot softmax, shift
 invariance under K mean smoothing, permutation equivariance), and library
 special cases (torch SDPA in float64, torch float8_e4m3fn casts).
 """
-from .attention import attention_fp64, attention_f64, widen_bf16, score_matrix_fp64  # noqa: F401
+from .attention import (attention_fp64, attention_f64, attention_varlen_fp64,  # noqa: F401
+                        score_matrix_fp64, widen_bf16)
 from . import quant8  # noqa: F401

@@ -12,7 +12,10 @@ oracle is the plain definition and nothing else.
 Readings of points the pages leave open (each is listed in the design notes):
   * GQA: query head h reads kv head floor(h / (Hq / Hkv)) (contiguous groups;
     the pages only name MQA, "FlashAttention-2 (2023)" section).
-  * Causal: key j is visible to query i iff j <= i; only Nq == Nkv is defined.
+  * Causal: key j is visible to query i iff j <= i + (Nkv - Nq) (aligned to
+    the bottom right, so the last query sees every key: a prefill whose first
+    Nkv - Nq keys are a cache). For Nq == Nkv this is j <= i. A row that sees
+    no key (possible only when Nq > Nkv) has O = 0 and LSE = -inf.
   * scale is an explicit argument (1/sqrt(d) by default in the binding).
   * LSE_i = ln sum_j exp(scale * S_raw_ij) over visible j, natural log,
     scale included.
@@ -52,10 +55,8 @@ def score_matrix_fp64(q: np.ndarray, k: np.ndarray, scale: float, causal: bool,
     idx = np.arange(Nq) if rows is None else np.asarray(rows)
     S = scale * (q[idx] @ k.T)
     if causal:
-        if Nq != Nkv:
-            raise ValueError("causal attention is defined here only for Nq == Nkv")
         j = np.arange(Nkv)
-        S = np.where(j[None, :] <= idx[:, None], S, -np.inf)
+        S = np.where(j[None, :] <= idx[:, None] + (Nkv - Nq), S, -np.inf)
     return S
 
 
@@ -99,14 +100,43 @@ def attention_f64(q, k, v, causal: bool, scale: float, rows=None, return_p: bool
             vh = widen(v[b, hk])
             r = None if rows is None else rows[b, h]
             S = score_matrix_fp64(qh, kh, scale, causal, r)
-            m = S.max(axis=1)                      # row maximum (finite: >= 1 visible key)
-            E = np.exp(S - m[:, None])             # exp(-inf) = 0 at masked keys
+            m = S.max(axis=1) if S.shape[1] else np.full(S.shape[0], -np.inf)
+            empty = np.isinf(m)                    # rows that see no key
+            m_safe = np.where(empty, 0.0, m)
+            E = np.exp(S - m_safe[:, None])        # exp(-inf) = 0 at masked keys
             l = E.sum(axis=1)
-            P = E / l[:, None]
+            with np.errstate(invalid="ignore", divide="ignore"):
+                P = np.where(empty[:, None], 0.0, E / np.where(empty, 1.0, l)[:, None])
+                L[b, h] = np.where(empty, -np.inf, m_safe + np.log(l))
             O[b, h] = P @ vh
-            L[b, h] = m + np.log(l)
             if return_p:
                 Ps[b, h] = P
     if return_p:
         return O, L, Ps
+    return O, L
+
+
+def attention_varlen_fp64(q_bits, k_bits, v_bits, cu_seqlens_q, cu_seqlens_k, causal: bool,
+                          scale: float):
+    """Packed variable-length attention: q_bits uint16 [total_q, Hq, d], k/v
+    [total_k, Hkv, d]; sequence s owns query rows cu_seqlens_q[s]:cu_seqlens_q[s+1]
+    and key rows cu_seqlens_k[s]:cu_seqlens_k[s+1], and attends only within
+    itself (causal masks are per sequence, bottom-right aligned).
+
+    Returns O float64 [total_q, Hq, d] and LSE float64 [Hq, total_q].
+    """
+    total_q, Hq, d = q_bits.shape
+    O = np.zeros((total_q, Hq, d))
+    L = np.full((Hq, total_q), -np.inf)
+    for s in range(len(cu_seqlens_q) - 1):
+        q0, q1 = int(cu_seqlens_q[s]), int(cu_seqlens_q[s + 1])
+        k0, k1 = int(cu_seqlens_k[s]), int(cu_seqlens_k[s + 1])
+        if q1 == q0:
+            continue
+        qs = np.ascontiguousarray(q_bits[q0:q1].transpose(1, 0, 2))[None]
+        ks = np.ascontiguousarray(k_bits[k0:k1].transpose(1, 0, 2))[None]
+        vs = np.ascontiguousarray(v_bits[k0:k1].transpose(1, 0, 2))[None]
+        Os, Ls = attention_fp64(qs, ks, vs, causal, scale)
+        O[q0:q1] = Os[0].transpose(1, 0, 2)
+        L[:, q0:q1] = Ls[0]
     return O, L
