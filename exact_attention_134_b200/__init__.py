@@ -42,6 +42,7 @@ _lock = threading.Lock()
 _c_int, _c_float, _vp, _sz = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 _SIGNATURES = {
     "attn_fwd": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp]),
+    "attn_fwd_varlen": (_c_int, [_vp] * 7 + [_c_int] * 8 + [_c_float, _vp]),
     "attn_fwd_host_buffer_size": (_sz, [_c_int] * 6),
     "attn_fwd_host": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp, _sz, _vp]),
     "attn_fwd_q8_workspace_size": (_sz, [_c_int] * 6),
@@ -121,6 +122,41 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None
                         B, Hq, Hkv, Nq, Nkv, d, int(bool(causal)), float(scale),
                         _stream_handle(q.device))
     _check(st, "attn_fwd")
+    return out, lse
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, causal: bool = False,
+                    scale: float | None = None, out=None, lse=None):
+    """Packed variable-length attention on the GPU.
+
+    q: bf16 cuda [total_q, Hq, d]; k, v: bf16 cuda [total_k, Hkv, d];
+    cu_seqlens_q / cu_seqlens_k: int32 cuda [num_seqs + 1] row offsets.
+    Returns (o bf16 [total_q, Hq, d], lse fp32 [Hq, total_q]).
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor [total, H, d]")
+    for name, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.dim() != 1:
+            raise ValueError(f"{name} must be a contiguous int32 CUDA vector")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both hold num_seqs + 1 offsets")
+    total_q, Hq, d = q.shape
+    total_k, Hkv, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or dk != d:
+        raise ValueError("shape mismatch between q and k/v")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    st = lib().attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                               cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(),
+                               cu_seqlens_q.numel() - 1, int(max_seqlen_q), total_q, total_k, Hq, Hkv, d,
+                               int(bool(causal)), float(scale), _stream_handle(q.device))
+    _check(st, "attn_fwd_varlen")
     return out, lse
 
 

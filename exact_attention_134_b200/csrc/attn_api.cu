@@ -80,7 +80,6 @@ attn_status_t check_args(const void* q, const void* k, const void* v, const void
   if (!std::isfinite(scale) || !(scale > 0.0f)) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if (causal && Nq != Nkv) return ATTN_ERR_UNSUPPORTED;
   if (B > 65535 || Hq > 65535) return ATTN_ERR_UNSUPPORTED;
   // TMA global strides must stay below 2^40 bytes.
   const unsigned long long head_bytes_q = 2ull * (unsigned long long)Nq * d;
@@ -97,6 +96,20 @@ bool make_map(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * (cuuint64_t)d * 2};
   cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t elem_strides[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                        strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Packed bf16 tensor [total, H, d] as {d, H, total}; box = 64 columns x 1 head x
+// 128 rows (the same shared-memory layout as the dense box).
+bool make_map_packed(CUtensorMap* m, const void* ptr, int d, int H, int total) {
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)total};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * (cuuint64_t)d * 2};
+  cuuint32_t box[3] = {64, 1, 128};
   cuuint32_t elem_strides[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
                         strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -131,6 +144,8 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.o = o;
   p.lse = lse;
   p.status = status;
+  p.cu_q = nullptr;
+  p.cu_k = nullptr;
   p.B = B;
   p.Nq = Nq;
   p.Nkv = Nkv;
@@ -150,6 +165,38 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
   return cuda_status(attn_sm100::launch_fwd_bf16(tq, tk, tv, to, p, d, stream));
+}
+
+attn_status_t run_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const int* cu_q, const int* cu_k, int num_seqs, int max_seqlen_q,
+                             int total_q, int total_k, int Hq, int Hkv, int d, int causal,
+                             float scale, cudaStream_t stream) {
+  int* status = device_status_ptr();
+  if (!status) return ATTN_ERR_CUDA;
+  alignas(64) CUtensorMap tq, tk, tv;
+  if (!make_map_packed(&tq, q, d, Hq, total_q) || !make_map_packed(&tk, k, d, Hkv, total_k) ||
+      !make_map_packed(&tv, v, d, Hkv, total_k))
+    return ATTN_ERR_CUDA;
+  attn_sm100::FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.status = status;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.B = num_seqs;
+  p.Nq = total_q;
+  p.Nkv = total_k;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.causal = causal;
+  const int rows = attn_sm100::fwd_rows_per_cta();
+  p.num_row_blocks = (max_seqlen_q + rows - 1) / rows;
+  p.num_units = 0;
+  p.num_ctas = 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = (unsigned long long)g_timeout_ns.load();
+  // the output map is unused by the packed path (rows are stored one by one)
+  return cuda_status(attn_sm100::launch_fwd_bf16(tq, tk, tv, tq, p, d, stream));
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -279,6 +326,22 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   if (s != ATTN_OK) return s;
   return run_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale,
                  static_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                              const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                              int max_seqlen_q, int total_q, int total_k, int Hq, int Hkv, int d,
+                              int causal, float scale, void* stream) {
+  if (!cu_seqlens_q || !cu_seqlens_k) return ATTN_ERR_INVALID_ARG;
+  if (num_seqs <= 0 || max_seqlen_q <= 0) return ATTN_ERR_INVALID_ARG;
+  // the dense checks with B = 1 cover pointers, sizes, heads, scale, d and alignment
+  attn_status_t s = check_args(q, k, v, o, lse, 1, Hq, Hkv, total_q, total_k, d, causal, scale);
+  if (s != ATTN_OK) return s;
+  if (num_seqs > 65535) return ATTN_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) | reinterpret_cast<uintptr_t>(cu_seqlens_k)) & 3u)
+    return ATTN_ERR_ALIGNMENT;
+  return run_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q,
+                        total_q, total_k, Hq, Hkv, d, causal, scale, static_cast<cudaStream_t>(stream));
 }
 
 size_t attn_fwd_host_buffer_size(int B, int Hq, int Hkv, int Nq, int Nkv, int d) {

@@ -107,7 +107,11 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
   }
 }
 
-template <int D>
+// VL = false: dense [B, H, N, d] tensors, one grid z-slice per batch entry.
+// VL = true : packed variable-length sequences [total, H, d]; grid z = sequence,
+//             its query/key rows come from cu_seqlens; O and LSE are stored
+//             row by row (a TMA box could cross into the next sequence).
+template <int D, bool VL>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -130,26 +134,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit: 256 query rows of one (batch, query head)
-  const int row_block = p.causal ? (p.num_row_blocks - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+  // ---- work unit: 256 query rows of one (sequence, query head)
+  int Lq = p.Nq, Lk = p.Nkv, q_start = 0, k_start = 0;
+  if (VL) {
+    const int sq = blockIdx.z;
+    q_start = min(max(p.cu_q[sq], 0), p.Nq);
+    Lq = min(max(p.cu_q[sq + 1], q_start), p.Nq) - q_start;
+    k_start = min(max(p.cu_k[sq], 0), p.Nkv);
+    Lk = min(max(p.cu_k[sq + 1], k_start), p.Nkv) - k_start;
+  }
+  const int nrb = (Lq + 2 * kBM - 1) / (2 * kBM);
+  if ((int)blockIdx.x >= nrb) return;  // this sequence has fewer rows (the whole CTA leaves)
+  const int row_block = p.causal ? (nrb - 1 - (int)blockIdx.x) : (int)blockIdx.x;
   const int hq = blockIdx.y;
-  const int b = blockIdx.z;
+  const int b = VL ? 0 : (int)blockIdx.z;
   const int hk = hq / (p.Hq / p.Hkv);
-  const int q0 = row_block * 2 * kBM;
+  const int q0 = row_block * 2 * kBM;  // first query row of the unit, within its sequence
   const int bh_q = b * p.Hq + hq;
   const int bh_kv = b * p.Hkv + hk;
-  // K/V tiles each query tile needs: all of them, or (causal) up to its last row;
-  // query tile 0 of a causal CTA skips the last tile, which it would see fully masked
-  int n_tiles, n_tiles0;
-  if (p.causal) {
-    const int last_row = min(q0 + 2 * kBM - 1, p.Nq - 1);
-    n_tiles = min(last_row, p.Nkv - 1) / kBN + 1;
-    const int last_row0 = min(q0 + kBM - 1, p.Nq - 1);
-    n_tiles0 = min(last_row0, p.Nkv - 1) / kBN + 1;
-  } else {
-    n_tiles = (p.Nkv + kBN - 1) / kBN;
-    n_tiles0 = n_tiles;
-  }
+  // causal mask aligned to the bottom right: key j is visible to query i iff
+  // j <= i + (Lk - Lq)
+  const int diag = p.causal ? Lk - Lq : 0;
+  // K/V tiles a query tile needs (at least one, so every pipeline runs; a row
+  // that sees no key ends with l = 0): all of them, or (causal) up to the key
+  // its last row sees. Query tile 0 of a causal CTA thus skips the last tile.
+  auto tiles_for = [&](int last_row) -> int {
+    if (!p.causal) return max(1, (Lk + kBN - 1) / kBN);
+    const int last_key = min(last_row + diag, Lk - 1);
+    return last_key < 0 ? 1 : last_key / kBN + 1;
+  };
+  const int n_tiles = tiles_for(min(q0 + 2 * kBM - 1, Lq - 1));
+  const int n_tiles0 = tiles_for(min(q0 + kBM - 1, Lq - 1));
+  // TMA coordinates (rows, outer) of a query tile / a K/V tile
+  const int q_c1 = VL ? hq : 0, kv_c1 = VL ? hk : 0;
+  auto q_row = [&](int t) { return VL ? q_start + q0 + t * kBM : q0 + t * kBM; };
+  auto kv_row = [&](int j) { return VL ? k_start + j * kBN : j * kBN; };
   const uint64_t budget = p.timeout_ns;
 
   // ---- setup: barriers (thread 0), TMEM (MMA warp)
@@ -193,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < 2; ++t)
         for (int bx = 0; bx < C::kBoxes; ++bx)
           tma_load_3d(sQ + t * C::kTileBytes + bx * kBoxBytes, &tm_q, bar(BarLayout::kQFull),
-                      bx * 64, q0 + t * kBM, bh_q);
+                      bx * 64, VL ? q_c1 : q_row(t), VL ? q_row(t) : bh_q);
     }
     for (int j = 0; j < n_tiles && ok; ++j) {
       for (int which = 0; which < 2; ++which) {  // 0 = K_j, 1 = V_j
@@ -206,8 +225,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(fb, C::kTileBytes);
           const CUtensorMap* tm = which ? &tm_v : &tm_k;
           for (int bx = 0; bx < C::kBoxes; ++bx)
-            tma_load_3d(sRing + stage * C::kTileBytes + bx * kBoxBytes, tm, fb, bx * 64, j * kBN,
-                        bh_kv);
+            tma_load_3d(sRing + stage * C::kTileBytes + bx * kBoxBytes, tm, fb, bx * 64,
+                        VL ? kv_c1 : kv_row(j), VL ? kv_row(j) : bh_kv);
         }
         __syncwarp();
         ++issued;
@@ -339,8 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // mask: keys >= Nkv, and (causal) keys after this row
       const int kv0 = j * kBN;
-      int lim = p.Nkv - kv0;
-      if (p.causal) lim = min(lim, row - kv0 + 1);
+      int lim = Lk - kv0;
+      if (p.causal) lim = min(lim, row + diag - kv0 + 1);
       if (lim < kBN) {
 #pragma unroll
         for (int c = 0; c < kBN; ++c)
@@ -394,7 +413,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (ok) ok = warp_all(bounded_wait(bar(BarLayout::kOFinal), 0, abort_flag, budget));
-    if (ok) {
+    if (ok && VL) {
+      // ---- epilogue (packed sequences): O = O_acc / l -> bf16 stored row by row
+      tc_fence_after();
+      const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+      const bool valid = row < Lq;  // q_start + row < total holds by the clamping above
+      uint4* const orow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) +
+                                                   ((size_t)(q_start + (valid ? row : 0)) * p.Hq + hq) * D);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * c, o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
+            orow[c * 4 + q] = v;
+          }
+        }
+      }
+      if (valid)  // LSE of packed sequences: [Hq, total_q]
+        p.lse[(size_t)hq * p.Nq + q_start + row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+    } else if (ok) {
       // ---- epilogue: O = O_acc / l -> bf16 into the (now free) Q_t buffer, then TMA store
       tc_fence_after();
       const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
@@ -419,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(BarLayout::kEpi + t));
-      if (row < p.Nq) p.lse[(size_t)bh_q * p.Nq + row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+      if (row < Lq) p.lse[(size_t)bh_q * p.Nq + row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
       if (r == 0) {
         volatile int no_abort = 0;
         if (bounded_wait(bar(BarLayout::kEpi + t), 0, &no_abort, budget)) {
@@ -449,21 +494,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 static int smem_bytes() { return FwdCfg<D>::kSmemBytes; }
 
-template <int D>
+template <int D, bool VL>
 static cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& to, const FwdParams& p, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_bf16_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_bf16_kernel<D, VL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<D>());
   if (e != cudaSuccess) return e;
-  dim3 grid(p.num_row_blocks, p.Hq, p.B);
-  attn_fwd_bf16_kernel<D><<<grid, kThreads, smem_bytes<D>(), stream>>>(tq, tk, tv, to, p);
+  dim3 grid(p.num_row_blocks, p.Hq, p.B);  // varlen: B = number of sequences
+  attn_fwd_bf16_kernel<D, VL><<<grid, kThreads, smem_bytes<D>(), stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t stream) {
-  if (d == 128) return launch_fwd_d<128>(tq, tk, tv, to, p, stream);
-  return launch_fwd_d<64>(tq, tk, tv, to, p, stream);
+  const bool vl = p.cu_q != nullptr;
+  if (d == 128)
+    return vl ? launch_fwd_d<128, true>(tq, tk, tv, to, p, stream)
+              : launch_fwd_d<128, false>(tq, tk, tv, to, p, stream);
+  return vl ? launch_fwd_d<64, true>(tq, tk, tv, to, p, stream)
+            : launch_fwd_d<64, false>(tq, tk, tv, to, p, stream);
 }
 
 int fwd_rows_per_cta() { return 2 * kBM; }

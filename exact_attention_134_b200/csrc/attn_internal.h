@@ -15,9 +15,11 @@ struct FwdParams {
   void* o;                        // bf16 [B, Hq, Nq, d]
   float* lse;                     // fp32 [B, Hq, Nq]
   int* status;                    // device status word: [0] code, [1] where
-  int B, Nq, Nkv, Hq, Hkv;
+  const int* cu_q;                // packed sequences: query row offsets [B + 1] (else null)
+  const int* cu_k;                //                   key row offsets [B + 1]
+  int B, Nq, Nkv, Hq, Hkv;        // packed: B = sequences, Nq / Nkv = total rows
   int causal;
-  int num_row_blocks;             // ceil(Nq / rows per work unit)
+  int num_row_blocks;             // ceil(Nq / rows per work unit); packed: of the longest sequence
   int num_units;                  // B * Hq * num_row_blocks
   int num_ctas;                   // persistent grid size (SM count)
   float scale_log2;               // scale * log2(e)

@@ -346,10 +346,14 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
   const int q0 = row_block * 2 * kTok;
   const int bh_q = b * p.Hq + hq;
   const int bh_kv = b * p.Hkv + hk;
+  // causal mask aligned to the bottom right: key j visible to query i iff
+  // j <= i + (Nkv - Nq); at least one K/V tile per unit (a row that sees no key
+  // ends with l = 0, O = 0, LSE = -inf)
+  const int diag = p.causal ? p.Nkv - p.Nq : 0;
   int n_tiles;
   if (p.causal) {
-    const int last_row = min(q0 + 2 * kTok - 1, p.Nq - 1);
-    n_tiles = min(last_row, p.Nkv - 1) / kTok + 1;
+    const int last_key = min(min(q0 + 2 * kTok - 1, p.Nq - 1) + diag, p.Nkv - 1);
+    n_tiles = last_key < 0 ? 1 : last_key / kTok + 1;
   } else {
     n_tiles = (p.Nkv + kTok - 1) / kTok;
   }
@@ -542,10 +546,10 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
       }
       const int kv0 = j * kTok;
       const bool tile_masked =
-          (kv0 + kTok > p.Nkv) || (p.causal && kv0 + kTok - 1 > q0 + t * kTok);
+          (kv0 + kTok > p.Nkv) || (p.causal && kv0 + kTok - 1 > q0 + t * kTok + diag);
       if (tile_masked) {
         int lim = p.Nkv - kv0;
-        if (p.causal) lim = min(lim, row - kv0 + 1);
+        if (p.causal) lim = min(lim, row + diag - kv0 + 1);
 #pragma unroll
         for (int c = 0; c < kTok; ++c)
           if (c >= lim) sr[c] = __float_as_uint(-INFINITY);

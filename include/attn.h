@@ -17,7 +17,10 @@
  *     scale included).
  *   - GQA: query head h reads kv head h / (Hq / Hkv) (contiguous groups; the
  *     pages name MQA only, "FlashAttention-2 (2023)" section). Hq % Hkv == 0.
- *   - Causal: key j is visible to query i iff j <= i; requires Nq == Nkv.
+ *   - Causal: key j is visible to query i iff j <= i + (Nkv - Nq), i.e. the
+ *     mask is aligned to the bottom right (for Nq == Nkv: j <= i; for Nq < Nkv
+ *     a prefill whose first Nkv - Nq keys are a cache). A row that sees no
+ *     key (only possible when Nq > Nkv) gets O = 0 and LSE = -inf.
  *   - Head dim d is 64 or 128.
  *   - Ownership: the caller owns every buffer; device pointers must stay valid
  *     until the work queued on `stream` has finished. The library allocates no
@@ -51,7 +54,7 @@ extern "C" {
 typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_INVALID_ARG = 1,  /* NULL pointer, a size <= 0, Hq % Hkv != 0, scale not finite or <= 0 */
-  ATTN_ERR_UNSUPPORTED = 2,  /* d not in {64, 128}; causal with Nq != Nkv; sizes beyond 2^31 elements per tensor dim */
+  ATTN_ERR_UNSUPPORTED = 2,  /* d not in {64, 128}; B, Hq or sequence count > 65535; a head beyond 2^40 bytes */
   ATTN_ERR_ALIGNMENT = 3,    /* a device pointer is not 16-byte aligned */
   ATTN_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (no device, launch failure, ...) */
   ATTN_ERR_TIMEOUT = 5,      /* a kernel pipeline wait exceeded its budget (reported by attn_get_status) */
@@ -65,12 +68,34 @@ typedef enum {
  *   o      device, bf16 [B, Hq, Nq, d]          (written; RNE from fp32)
  *   lse    device, fp32 [B, Hq, Nq]             (written)
  *   scale  softmax scale applied to Q K^T (typically 1/sqrt(d)); finite, > 0
- *   causal 0 = full attention, 1 = lower-triangular mask (needs Nq == Nkv)
+ *   causal 0 = full attention, 1 = causal mask aligned to the bottom right
  * Allocates nothing; one kernel launch on `stream`.
  */
 ATTN_API attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                        int B, int Hq, int Hkv, int Nq, int Nkv, int d,
                        int causal, float scale, void* stream);
+
+/*
+ * attn_fwd_varlen — the same operation on packed variable-length sequences
+ * (a batch of prompts of different lengths without padding). Sequence s owns
+ * query rows cu_seqlens_q[s] .. cu_seqlens_q[s+1]-1 and key/value rows
+ * cu_seqlens_k[s] .. cu_seqlens_k[s+1]-1 and attends only within itself; the
+ * causal mask is per sequence, aligned to the bottom right.
+ *   q, o           device, bf16 [total_q, Hq, d]        (o written)
+ *   k, v           device, bf16 [total_k, Hkv, d]
+ *   lse            device, fp32 [Hq, total_q]           (written)
+ *   cu_seqlens_q/k device, int32 [num_seqs + 1], non-decreasing, starting at 0
+ *                  and ending at total_q / total_k (caller's responsibility;
+ *                  offsets outside [0, total] are clamped, never followed)
+ *   max_seqlen_q   >= the longest query sequence (sizes the grid; rows beyond
+ *                  it are not computed)
+ * Allocates nothing; one kernel launch on `stream`.
+ */
+ATTN_API attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void* o,
+                                       float* lse, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                                       int num_seqs, int max_seqlen_q, int total_q, int total_k,
+                                       int Hq, int Hkv, int d, int causal, float scale,
+                                       void* stream);
 
 /*
  * attn_fwd_host — the same operation on HOST buffers, for callers whose data
