@@ -29,7 +29,8 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synthetic import WORKLOADS, Workload, bf16_bits, make_qkv  # noqa: E402
+from synthetic import (VARLEN_WORKLOADS, WORKLOADS, Workload, bf16_bits, make_qkv,  # noqa: E402
+                       make_varlen)
 
 HEADLINE = "outlier_8k_causal"
 EXTRA_BF16 = ["causal_2k_d128", "outlier_8k_full", "gqa_32k_d128", "gqa_32k_d64"]
@@ -266,6 +267,32 @@ def bench_q8(w: Workload, steps: int, warmup: int, world: int, rank: int, lib_mo
     return full_ms, pre_ms
 
 
+def bench_varlen(name: str, steps: int, warmup: int, world: int, lib_mod):
+    """Packed variable-length prefill (inputs larger than L2)."""
+    import torch
+    w = VARLEN_WORKLOADS[name]
+    q, k, v, cu = make_varlen(w)
+    qd, kd, vd, cud = q.cuda(), k.cuda(), v.cuda(), cu.cuda()
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.Hq, q.shape[0]), dtype=torch.float32, device="cuda")
+    max_len = max(w.lengths())
+
+    def step():
+        lib_mod.attn_fwd_varlen(qd, kd, vd, cud, cud, max_len, causal=w.causal, out=o, lse=lse)
+
+    _barrier(world)
+    times = time_device(step, steps, max(warmup, 3))
+    _barrier(world)
+    st, where = lib_mod.get_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} at {where:#x}")
+    ms = _max_over_ranks(statistics.mean(times), world)
+    return {"tflops": round(world * w.flops / (ms * 1e-3) / 1e12, 1), "ms_per_step": round(ms, 4),
+            "sequences": w.num_seqs, "total_tokens": int(q.shape[0]),
+            "lengths": f"log-uniform in [{w.min_len}, {w.max_len}], seed {w.seed}",
+            "l2": "inputs_larger_than_l2"}
+
+
 def bench_e2e(w: Workload, steps: int, warmup: int, world: int, rank: int, lib_mod):
     """Same metric through the host-buffer entry point: every step copies the
     step's inputs from pinned host memory and reads O and LSE back."""
@@ -357,6 +384,9 @@ def run_ours(args):
                             "l2": r["l2"]}
             del r
             torch.cuda.empty_cache()
+        extras["varlen_prefill_mixed"] = bench_varlen("varlen_prefill_mixed", max(3, args.steps // 2),
+                                                      3, world, attn)
+        torch.cuda.empty_cache()
         wq = WORKLOADS["q8_8k_outlier"]
         full_ms, pre_ms = bench_q8(wq, max(3, args.steps // 2), 3, world, rank, attn)
         fp8_peak = 2.0 * peaks["bf16"]

@@ -48,6 +48,8 @@ _SIGNATURES = {
     "attn_fwd_q8_workspace_size": (_sz, [_c_int] * 6),
     "attn_fwd_q8": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp, _sz, _vp]),
     "attn_q8_prepass": (_c_int, [_vp, _vp, _vp] + [_c_int] * 6 + [_vp, _sz, _vp]),
+    "attn_fwd_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp, _sz, _vp]),
+    "attn_fp8_prepass": (_c_int, [_vp, _vp, _vp] + [_c_int] * 6 + [_vp, _sz, _vp]),
     "attn_q8_workspace_offsets": (_c_int, [_c_int] * 6 + [ctypes.POINTER(_sz)]),
     "attn_get_status": (_c_int, [_vp]),
     "attn_get_status_ex": (_c_int, [_vp, ctypes.POINTER(_c_int)]),
@@ -173,8 +175,9 @@ def q8_workspace_offsets(B, Hq, Hkv, Nq, Nkv, d) -> list[int]:
 
 
 def attn_fwd_q8(q, k, v, causal: bool = False, scale: float | None = None, workspace=None,
-                out=None, lse=None):
-    """8-bit (INT8 Q K^T after K smoothing, FP8 P V) attention forward.
+                out=None, lse=None, qk_format: str = "int8"):
+    """8-bit attention forward: INT8 Q K^T after K smoothing (``qk_format="int8"``)
+    or FP8 e4m3 Q K^T with block scales and no smoothing (``"fp8"``); FP8 P V.
 
     Same tensors as ``attn_fwd``; ``workspace`` is a uint8 cuda tensor of at
     least ``q8_workspace_size`` bytes (allocated here if None). Returns (o, lse).
@@ -193,19 +196,23 @@ def attn_fwd_q8(q, k, v, causal: bool = False, scale: float | None = None, works
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
-    st = lib().attn_fwd_q8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                           B, Hq, Hkv, Nq, Nkv, d, int(bool(causal)), float(scale),
-                           workspace.data_ptr(), workspace.numel(), _stream_handle(q.device))
-    _check(st, "attn_fwd_q8")
+    if qk_format not in ("int8", "fp8"):
+        raise ValueError("qk_format must be 'int8' or 'fp8'")
+    fn = lib().attn_fwd_q8 if qk_format == "int8" else lib().attn_fwd_fp8
+    st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+            B, Hq, Hkv, Nq, Nkv, d, int(bool(causal)), float(scale),
+            workspace.data_ptr(), workspace.numel(), _stream_handle(q.device))
+    _check(st, "attn_fwd_q8" if qk_format == "int8" else "attn_fwd_fp8")
     return out, lse
 
 
-def q8_prepass(q, k, v, workspace):
+def q8_prepass(q, k, v, workspace, qk_format: str = "int8"):
     """Run only the 8-bit prepass (K mean, scales, quantisation) into ``workspace``."""
     B, Hq, Hkv, Nq, Nkv, d = _shape_args(q, k, v)
-    st = lib().attn_q8_prepass(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, Nq, Nkv, d,
-                               workspace.data_ptr(), workspace.numel(), _stream_handle(q.device))
-    _check(st, "attn_q8_prepass")
+    fn = lib().attn_q8_prepass if qk_format == "int8" else lib().attn_fp8_prepass
+    st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, Nq, Nkv, d,
+            workspace.data_ptr(), workspace.numel(), _stream_handle(q.device))
+    _check(st, "8-bit prepass")
 
 
 def host_buffer_size(B, Hq, Hkv, Nq, Nkv, d) -> int:

@@ -224,7 +224,7 @@ void q8_layout(int B, int Hq, int Hkv, int Nq, int Nkv, int d, size_t off[kQ8Reg
 attn_status_t run_q8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
                      void* workspace, size_t workspace_bytes, bool prepass_only,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, bool fp8_qk = false) {
   if (!workspace || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
   size_t off[kQ8Regions + 1];
   q8_layout(B, Hq, Hkv, Nq, Nkv, d, off);
@@ -246,6 +246,7 @@ attn_status_t run_q8(const void* q, const void* k, const void* v, void* o, float
   L.B = B;
   L.Hkv = Hkv;
   L.prepass_only = prepass_only;
+  L.fp8_qk = fp8_qk;
   attn_sm100::Q8Params& p = L.p;
   p.lse = lse;
   p.status = status;
@@ -411,6 +412,24 @@ attn_status_t attn_q8_prepass(const void* q, const void* k, const void* v, int B
   if (s != ATTN_OK) return s;
   return run_q8(q, k, v, nullptr, nullptr, B, Hq, Hkv, Nq, Nkv, d, 0, 1.0f, workspace,
                 workspace_bytes, true, static_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                           int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  if (s != ATTN_OK) return s;
+  return run_q8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, workspace,
+                workspace_bytes, false, static_cast<cudaStream_t>(stream), true);
+}
+
+attn_status_t attn_fp8_prepass(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
+                               int Nq, int Nkv, int d, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  attn_status_t s = check_args(q, k, v, q, q, B, Hq, Hkv, Nq, Nkv, d, 0, 1.0f);
+  if (s != ATTN_OK) return s;
+  return run_q8(q, k, v, nullptr, nullptr, B, Hq, Hkv, Nq, Nkv, d, 0, 1.0f, workspace,
+                workspace_bytes, true, static_cast<cudaStream_t>(stream), true);
 }
 
 attn_status_t attn_get_status_ex(void* stream, int* where) {

@@ -58,6 +58,7 @@ struct Q8Launch {
   float* vmax_part;
   int B, Hkv;
   bool prepass_only;
+  bool fp8_qk;                    // e4m3 Q and K with block scales, no smoothing
 };
 
 cudaError_t launch_q8(const Q8Launch& L, int d, cudaStream_t stream);

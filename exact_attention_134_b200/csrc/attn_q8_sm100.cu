@@ -137,7 +137,8 @@ __global__ void __launch_bounds__(kPrepThreads)
 }
 
 // ----------------------------------------------------------------- prepass 2
-template <int D>
+// F8 = true (FP8 Q K^T with block scales, no smoothing): kbar is zero.
+template <int D, bool F8>
 __global__ void q8_kv_final_kernel(const double* __restrict__ ksum_part,
                                    const float* __restrict__ vmax_part, int Nkv, int nkb,
                                    float* __restrict__ kbar, float* __restrict__ sv) {
@@ -149,12 +150,32 @@ __global__ void q8_kv_final_kernel(const double* __restrict__ ksum_part,
     acc += ksum_part[(bh * nkb + i) * D + c];
     m = fmaxf(m, vmax_part[(bh * nkb + i) * D + c]);
   }
-  kbar[bh * D + c] = static_cast<float>(acc / static_cast<double>(Nkv));
+  kbar[bh * D + c] = F8 ? 0.0f : static_cast<float>(acc / static_cast<double>(Nkv));
   sv[bh * D + c] = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
 }
 
 // ----------------------------------------------------------------- prepass 3
-template <int D>
+// Packs 8 codes of x / s (quotients rounded to nearest): INT8 (round half to
+// even, clamped to +-127) or, with F8, e4m3 (round to nearest even, saturating).
+template <bool F8>
+__device__ __forceinline__ uint2 codes8(const float (&x)[8], float s, float r) {
+  if (F8) {
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = div_rn(x[i], s, r);
+    return make_uint2(pack_e4m3x2(y[0], y[1]) | (pack_e4m3x2(y[2], y[3]) << 16),
+                      pack_e4m3x2(y[4], y[5]) | (pack_e4m3x2(y[6], y[7]) << 16));
+  }
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    lo |= (uint32_t)(uint8_t)quant_i8(x[i], s, r) << (8 * i);
+    hi |= (uint32_t)(uint8_t)quant_i8(x[i + 4], s, r) << (8 * i);
+  }
+  return make_uint2(lo, hi);
+}
+
+template <int D, bool F8>
 __global__ void __launch_bounds__(kPrepThreads)
     q8_quantize_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                        const uint16_t* __restrict__ v, int B, int Hq, int Hkv, int Nq, int Nkv,
@@ -189,7 +210,7 @@ __global__ void __launch_bounds__(kPrepThreads)
       for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[pp][i]));
     }
     amax = block_max256(amax, red);
-    const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 1.0f;
+    const float s = amax > 0.0f ? __fdiv_rn(amax, F8 ? 448.0f : 127.0f) : 1.0f;
     const float r_q = __frcp_rn(s);
     float kb[8];
 #pragma unroll
@@ -203,13 +224,7 @@ __global__ void __launch_bounds__(kPrepThreads)
 #pragma unroll
       for (int o = VPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
       if (t < Nq) {
-        uint32_t lo = 0, hi = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          lo |= (uint32_t)(uint8_t)quant_i8(x[pp][i], s, r_q) << (8 * i);
-          hi |= (uint32_t)(uint8_t)quant_i8(x[pp][i + 4], s, r_q) << (8 * i);
-        }
-        *reinterpret_cast<uint2*>(q8 + ((size_t)bh * Nq + t) * D + vc * 8) = make_uint2(lo, hi);
+        *reinterpret_cast<uint2*>(q8 + ((size_t)bh * Nq + t) * D + vc * 8) = codes8<F8>(x[pp], s, r_q);
         if (vc == 0) qk[(size_t)bh * Nq + t] = dot;
       }
     }
@@ -241,19 +256,13 @@ __global__ void __launch_bounds__(kPrepThreads)
       for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[pp][i]));
     }
     amax = block_max256(amax, red);
-    const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 1.0f;
+    const float s = amax > 0.0f ? __fdiv_rn(amax, F8 ? 448.0f : 127.0f) : 1.0f;
     const float r_s = __frcp_rn(s);
 #pragma unroll
     for (int pp = 0; pp < NP; ++pp) {
       const int t = kb_i * kTok + rs + pp * RPP;
       if (t < Nkv) {
-        uint32_t lo = 0, hi = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          lo |= (uint32_t)(uint8_t)quant_i8(x[pp][i], s, r_s) << (8 * i);
-          hi |= (uint32_t)(uint8_t)quant_i8(x[pp][i + 4], s, r_s) << (8 * i);
-        }
-        *reinterpret_cast<uint2*>(k8 + (bh * Nkv + t) * D + vc * 8) = make_uint2(lo, hi);
+        *reinterpret_cast<uint2*>(k8 + (bh * Nkv + t) * D + vc * 8) = codes8<F8>(x[pp], s, r_s);
         float vf[8];
         unpack8(*reinterpret_cast<const uint4*>(v + (bh * Nkv + t) * D + vc * 8), vf);
         float y[8];
@@ -298,14 +307,18 @@ __device__ __forceinline__ void q8_flag_abort(volatile int* abort_flag, int* sta
 
 __device__ __forceinline__ bool q8_warp_all(bool v) { return __all_sync(0xffffffffu, v) != 0; }
 
-template <int D>
+// S = Q8 K8^T: INT8 (s32 accumulation) or, with F8, e4m3 (fp32 accumulation).
+template <int D, bool F8>
 __device__ __forceinline__ void issue_qk_i8(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
-  constexpr uint32_t idesc = idesc_s8_s32(128, 128);
+  constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(128, 128) : idesc_s8_s32(128, 128);
 #pragma unroll
   for (int kk = 0; kk < D / 32; ++kk) {
     const uint64_t a = smem_desc_sw(q_smem + kk * 32, 16, 8 * D, D);
     const uint64_t b = smem_desc_sw(k_smem + kk * 32, 16, 8 * D, D);
-    mma_i8_ss(d_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+    if (F8)
+      mma_f8_ss(d_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+    else
+      mma_i8_ss(d_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -320,7 +333,7 @@ __device__ __forceinline__ void issue_pv_f8(uint32_t o_tmem, uint32_t p_tmem, ui
   }
 }
 
-template <int D>
+template <int D, bool F8>
 __global__ void __launch_bounds__(kQ8Threads, 1)
     attn_fwd_q8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -453,7 +466,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
       }
       tc_fence_after();
       if (lane == 0) {
-        issue_qk_i8<D>(tS[0], q_smem[0], k_smem);
+        issue_qk_i8<D, F8>(tS[0], q_smem[0], k_smem);
         tc_commit(bar(Q8Bar::kSFull + 0));
       }
       __syncwarp();
@@ -467,7 +480,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
         }
       }
       if (lane == 0) {
-        issue_qk_i8<D>(tS[1], q_smem[1], k_smem);
+        issue_qk_i8<D, F8>(tS[1], q_smem[1], k_smem);
         tc_commit(bar(Q8Bar::kSFull + 1));
         tc_commit(bar(Q8Bar::kEmpty + k_stage));
       }
@@ -535,9 +548,10 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
       const float f = sq_t * p.sk[(size_t)bh_kv * p.nkb + j] * p.scale_log2;
       // s32 -> fp32 without the conversion unit: |s| <= 127 * 127 * d < 2^22, so
       // the bits of (s + 0x4B400000) are the float 1.5 * 2^23 + s exactly
+      // (the e4m3 MMA already accumulates in fp32)
       constexpr float kMagic = 12582912.0f;
 #pragma unroll
-      for (int c = 0; c < kTok; c += 2) {
+      for (int c = 0; c < (F8 ? 0 : kTok); c += 2) {
         const float2 v = add2(make_float2(__uint_as_float(sr[c] + 0x4B400000u),
                                           __uint_as_float(sr[c + 1] + 0x4B400000u)),
                               make_float2(-kMagic, -kMagic));
@@ -674,7 +688,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
   }
 }
 
-template <int D>
+template <int D, bool F8>
 cudaError_t launch_q8_d(const Q8Launch& L, cudaStream_t stream) {
   const int nqb = L.p.nqb, nkb = L.p.nkb;
   dim3 g1(nkb, L.Hkv, L.B);
@@ -682,28 +696,30 @@ cudaError_t launch_q8_d(const Q8Launch& L, cudaStream_t stream) {
       static_cast<const uint16_t*>(L.k), static_cast<const uint16_t*>(L.v), L.p.Nkv, nkb,
       L.ksum_part, L.vmax_part);
   dim3 g2(L.Hkv, L.B);
-  q8_kv_final_kernel<D><<<g2, D, 0, stream>>>(L.ksum_part, L.vmax_part, L.p.Nkv, nkb, L.kbar,
+  q8_kv_final_kernel<D, F8><<<g2, D, 0, stream>>>(L.ksum_part, L.vmax_part, L.p.Nkv, nkb, L.kbar,
                                               const_cast<float*>(L.p.sv));
   const long long tiles = (long long)L.B * L.p.Hq * nqb + (long long)L.B * L.Hkv * nkb;
-  q8_quantize_kernel<D><<<(unsigned)tiles, kPrepThreads, 0, stream>>>(
+  q8_quantize_kernel<D, F8><<<(unsigned)tiles, kPrepThreads, 0, stream>>>(
       static_cast<const uint16_t*>(L.q), static_cast<const uint16_t*>(L.k),
       static_cast<const uint16_t*>(L.v), L.B, L.p.Hq, L.Hkv, L.p.Nq, L.p.Nkv, nqb, nkb, L.kbar,
       L.p.sv, L.q8, L.k8, L.v8, const_cast<float*>(L.p.sq), const_cast<float*>(L.p.sk),
       const_cast<float*>(L.p.qk));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || L.prepass_only) return e;
-  e = cudaFuncSetAttribute(attn_fwd_q8_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(attn_fwd_q8_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Q8Cfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(L.p.num_row_blocks, L.p.Hq, L.B);
-  attn_fwd_q8_kernel<D><<<grid, kQ8Threads, Q8Cfg<D>::kSmemBytes, stream>>>(L.tq, L.tk, L.tv, L.to, L.p);
+  attn_fwd_q8_kernel<D, F8><<<grid, kQ8Threads, Q8Cfg<D>::kSmemBytes, stream>>>(L.tq, L.tk, L.tv, L.to, L.p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_q8(const Q8Launch& L, int d, cudaStream_t stream) {
-  return d == 128 ? launch_q8_d<128>(L, stream) : launch_q8_d<64>(L, stream);
+  if (L.fp8_qk)
+    return d == 128 ? launch_q8_d<128, true>(L, stream) : launch_q8_d<64, true>(L, stream);
+  return d == 128 ? launch_q8_d<128, false>(L, stream) : launch_q8_d<64, false>(L, stream);
 }
 
 }  // namespace attn_sm100

@@ -137,6 +137,25 @@ ATTN_API attn_status_t attn_fwd_q8(const void* q, const void* k, const void* v, 
                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_fwd_fp8 — the 8-bit forward with FP8 e4m3 Q and K instead of INT8 and
+ * no K smoothing, in the manner "Makale Bülteni — FlashAttention-3" ("İddia
+ * ve Gerçeklik") describes for its FP8 mode: block-wise dynamic scaling, one
+ * fp32 scale = amax / 448 per 128-token block of Q and of K; S = Q8 K8^T on
+ * FP8 tensor cores with fp32 accumulation; P and V exactly as in attn_fwd_q8.
+ * It is the comparison point for INT8 with K smoothing on channels with
+ * outliers. Same arguments, workspace and errors as attn_fwd_q8 (the workspace
+ * regions hold e4m3 codes for Q and K, kbar and q.kbar are zero).
+ * attn_fp8_prepass runs only its three prepass launches.
+ */
+ATTN_API attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                                    int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                                    int causal, float scale,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+ATTN_API attn_status_t attn_fp8_prepass(const void* q, const void* k, const void* v,
+                                        int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * attn_fwd_q8_noalloc — attn_fwd_q8 for callers that cannot allocate device
  * memory, e.g. a plugin inside another framework's inference engine that is
  * handed only its input and output buffers, or a program that must not call

@@ -115,6 +115,27 @@ def quant_int8_blocks(x: np.ndarray, block: int = BLOCK):
     return codes, scales
 
 
+def quant_e4m3_blocks(x: np.ndarray, block: int = BLOCK):
+    """Per-(b, h, 128-token block) FP8 e4m3 quantisation in float32 (block-wise
+    dynamic scaling in the FlashAttention-3 manner: scale = fp32(amax / 448),
+    amax = 0 -> 1; code = e4m3(fp32(x / scale))).
+
+    Returns (codes uint8 [B, H, N, d], scales float32 [B, H, ceil(N / block)]).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    B, H, N, d = x.shape
+    nb = -(-N // block)
+    codes = np.empty((B, H, N, d), dtype=np.uint8)
+    scales = np.empty((B, H, nb), dtype=np.float32)
+    for i in range(nb):
+        blk = x[:, :, i * block:(i + 1) * block, :]
+        amax = np.abs(blk).max(axis=(2, 3)).astype(np.float32)
+        s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+        codes[:, :, i * block:(i + 1) * block, :] = e4m3_encode((blk / s[:, :, None, None]).astype(np.float32))
+        scales[:, :, i] = s
+    return codes, scales
+
+
 def quant_v_fp8(v_bits: np.ndarray):
     """Per-(b, hkv, channel) FP8 e4m3 quantisation of V.
 
@@ -177,4 +198,35 @@ def sage8_attention_fp64(q_bits, k_bits, v_bits, causal: bool, scale: float, row
             Vd = e4m3_decode(v8[b, hk]) * sv[b, hk][None, :].astype(np.float64)
             O[b, h] = (P8 @ Vd) / (E4M3_MAX * l[:, None])
             L[b, h] = m + np.log(l) + scale * qk[b, h, idx]
+    return O, L
+
+
+def fp8qk_attention_fp64(q_bits, k_bits, v_bits, causal: bool, scale: float, rows=None):
+    """The FP8-Q K^T variant as a one-shot computation: e4m3 Q and K with one
+    scale per 128-token block and no smoothing, P and V as in
+    ``sage8_attention_fp64`` (P encoded relative to the exact row maximum)."""
+    B, Hq, Nq, d = q_bits.shape
+    Hkv, Nkv = k_bits.shape[1], k_bits.shape[2]
+    q8, sq = quant_e4m3_blocks(widen_bf16(q_bits).astype(np.float32))
+    k8, sk = quant_e4m3_blocks(widen_bf16(k_bits).astype(np.float32))
+    v8, sv = quant_v_fp8(v_bits)
+    R = Nq if rows is None else rows.shape[-1]
+    O = np.empty((B, Hq, R, d))
+    L = np.empty((B, Hq, R))
+    for b in range(B):
+        for h in range(Hq):
+            hk = _kv_head(h, Hq, Hkv)
+            idx = np.arange(Nq) if rows is None else rows[b, h]
+            qi = e4m3_decode(q8[b, h, idx]) * sq[b, h, idx // BLOCK][:, None].astype(np.float64)
+            kj = e4m3_decode(k8[b, hk]) * sk[b, hk, np.arange(Nkv) // BLOCK][:, None].astype(np.float64)
+            S = scale * (qi @ kj.T)
+            if causal:
+                S = np.where(np.arange(Nkv)[None, :] <= idx[:, None] + (Nkv - Nq), S, -np.inf)
+            m = S.max(axis=1)
+            E = np.exp(S - m[:, None])
+            l = E.sum(axis=1)
+            P8 = e4m3_decode(e4m3_encode((E * E4M3_MAX).astype(np.float32)))
+            Vd = e4m3_decode(v8[b, hk]) * sv[b, hk][None, :].astype(np.float64)
+            O[b, h] = (P8 @ Vd) / (E4M3_MAX * l[:, None])
+            L[b, h] = m + np.log(l)
     return O, L

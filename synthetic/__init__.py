@@ -132,3 +132,47 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """The raw bf16 bit patterns of a CPU tensor, as a uint16 numpy array."""
     assert t.dtype == torch.bfloat16 and t.device.type == "cpu"
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+@dataclasses.dataclass(frozen=True)
+class VarlenWorkload:
+    """A batch of prompts of different lengths, packed without padding."""
+    name: str
+    num_seqs: int
+    min_len: int
+    max_len: int
+    Hq: int
+    Hkv: int
+    d: int
+    causal: bool
+    seed: int
+
+    def lengths(self) -> list[int]:
+        """Seeded log-uniform lengths in [min_len, max_len]."""
+        g = torch.Generator("cpu").manual_seed(self.seed)
+        u = torch.rand(self.num_seqs, generator=g, dtype=torch.float64)
+        lo, hi = math.log(self.min_len), math.log(self.max_len)
+        return [int(round(math.exp(lo + float(x) * (hi - lo)))) for x in u]
+
+    @property
+    def flops(self) -> float:
+        f = sum(4.0 * self.Hq * L * L * self.d for L in self.lengths())
+        return f / 2.0 if self.causal else f
+
+
+VARLEN_WORKLOADS = {
+    "varlen_prefill_mixed": VarlenWorkload("varlen_prefill_mixed", 16, 256, 8192, 32, 8, 128, True, 1007),
+}
+
+
+def make_varlen(w: VarlenWorkload):
+    """Packed q [total, Hq, d], k, v [total, Hkv, d] (bf16, CPU) and int32
+    cu_seqlens [num_seqs + 1] (the same offsets for queries and keys)."""
+    lens = w.lengths()
+    total = sum(lens)
+    g = torch.Generator("cpu").manual_seed(w.seed + 1)
+    q = torch.randn((total, w.Hq, w.d), generator=g, dtype=torch.float32)
+    k = torch.randn((total, w.Hkv, w.d), generator=g, dtype=torch.float32)
+    v = torch.randn((total, w.Hkv, w.d), generator=g, dtype=torch.float32)
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
+    return _bf16(q), _bf16(k), _bf16(v), cu

@@ -136,3 +136,67 @@ def test_q8_workspace_errors():
     with pytest.raises(attn.AttnError) as e:
         attn.attn_fwd_q8(q, k, v, workspace=small)
     assert e.value.status == 6
+
+
+# ---------------------------------------------------------------------------
+# FP8 e4m3 Q K^T with block-wise scaling (no smoothing)
+# ---------------------------------------------------------------------------
+def _check_prepass_fp8(B, Hq, Hkv, Nq, Nkv, d, seed, dist="normal"):
+    q, k, v = make_qkv(B, Hq, Hkv, Nq, Nkv, d, seed, dist)
+    ws = torch.empty(attn.q8_workspace_size(B, Hq, Hkv, Nq, Nkv, d), dtype=torch.uint8, device="cuda")
+    attn.q8_prepass(q.cuda(), k.cuda(), v.cuda(), ws, qk_format="fp8")
+    assert attn.get_status()[0] == 0
+    g = _regions(ws.cpu().numpy(), attn.q8_workspace_offsets(B, Hq, Hkv, Nq, Nkv, d), B, Hq, Hkv, Nq, Nkv, d)
+    qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
+    q8, sq = oq8.quant_e4m3_blocks(oracle.widen_bf16(qb).astype(np.float32))
+    k8, sk = oq8.quant_e4m3_blocks(oracle.widen_bf16(kb).astype(np.float32))
+    v8, sv = oq8.quant_v_fp8(vb)
+    assert np.all(g["kbar"] == 0.0) and np.all(g["qk"] == 0.0)
+    assert np.array_equal(g["sq"].view(np.uint32), sq.view(np.uint32))
+    assert np.array_equal(g["sk"].view(np.uint32), sk.view(np.uint32))
+    assert np.array_equal(g["q8"].view(np.uint8), q8)
+    assert np.array_equal(g["k8"].view(np.uint8), k8)
+    assert np.array_equal(g["v8"], v8)
+    assert np.array_equal(g["sv"].view(np.uint32), sv.view(np.uint32))
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 2, 300, 300, 128), (2, 4, 2, 257, 513, 64)])
+def test_fp8_prepass_bit_exact(shape):
+    _check_prepass_fp8(*shape, seed=sum(shape), dist="outlier_k")
+
+
+def _cos(a, b):
+    return float((a * b).sum() / math.sqrt((a * a).sum() * (b * b).sum()))
+
+
+@pytest.mark.parametrize("dist", ["normal", "outlier_k"])
+def test_fp8_forward_matches_its_method(dist):
+    # the FP8 Q K^T method is less accurate than INT8 with smoothing (3
+    # mantissa bits); the GPU must reproduce the method's own accuracy, i.e.
+    # stay as close to the exact result as the one-shot quantised oracle does
+    B, Hq, Hkv, N, d = 1, 4, 2, 1024, 128
+    q, k, v = make_qkv(B, Hq, Hkv, N, N, d, seed=21, dist=dist)
+    o, lse = attn.attn_fwd_q8(q.cuda(), k.cuda(), v.cuda(), causal=True, qk_format="fp8")
+    assert attn.get_status()[0] == 0
+    qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
+    sc = 1 / math.sqrt(d)
+    O, L = oracle.attention_fp64(qb, kb, vb, True, sc)
+    Of, Lf = oq8.fp8qk_attention_fp64(qb, kb, vb, True, sc)
+    og = o.cpu().float().numpy().astype(np.float64)
+    assert np.all(np.isfinite(og))
+    assert _cos(og, O) >= _cos(Of, O) - 1e-3
+    assert np.abs(og - Of).max() <= 5e-2  # GPU vs the method's one-shot result
+    assert np.abs(lse.cpu().numpy() - Lf).max() <= 5e-2
+
+
+def test_int8_smoothing_beats_fp8_on_outlier_channels():
+    B, Hq, Hkv, N, d = 1, 4, 2, 1024, 128
+    q, k, v = make_qkv(B, Hq, Hkv, N, N, d, seed=22, dist="outlier_k")
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    o8, l8 = attn.attn_fwd_q8(qc, kc, vc, causal=True, qk_format="int8")
+    of, lf = attn.attn_fwd_q8(qc, kc, vc, causal=True, qk_format="fp8")
+    O, L = oracle.attention_fp64(bf16_bits(q), bf16_bits(k), bf16_bits(v), True, 1 / math.sqrt(d))
+    c8 = _cos(o8.cpu().float().numpy().astype(np.float64), O)
+    cf = _cos(of.cpu().float().numpy().astype(np.float64), O)
+    assert c8 >= 0.999 and c8 > cf
+    assert np.abs(l8.cpu().numpy() - L).max() < np.abs(lf.cpu().numpy() - L).max()

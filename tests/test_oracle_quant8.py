@@ -120,3 +120,36 @@ def test_sage8_one_shot_within_8bit_tolerance(dist):
     vmax = np.abs(oracle.widen_bf16(vb)).max()
     assert np.max(np.abs(O - O8)) <= vmax * 2.0 ** -4 * 1.5
     assert np.max(np.abs(L - L8)) <= 5e-2
+
+
+def test_e4m3_block_quantisation_bounds():
+    rng = np.random.default_rng(2)
+    x = (rng.normal(size=(1, 2, 200, 32)) * rng.uniform(0.1, 30, size=(1, 2, 1, 1))).astype(np.float32)
+    x[0, 1, :128] = 0.0
+    codes, s = q8.quant_e4m3_blocks(x)
+    assert s[0, 1, 0] == 1.0 and np.all(codes[0, 1, :128] == 0)
+    deq = q8.e4m3_decode(codes) * np.repeat(s, 128, axis=2)[:, :, :200, None]
+    for h in range(2):
+        for i in range(2):
+            blk = x[0, h, i * 128:(i + 1) * 128]
+            if np.abs(blk).max() == 0:
+                continue
+            # the block maximum encodes to exactly 448 * scale
+            assert np.isclose(np.abs(deq[0, h, i * 128:(i + 1) * 128]).max(), np.abs(blk).max(), rtol=1e-6)
+            # relative error <= 2^-4 in the normal range, plus the subnormal quantum
+            err = np.abs(deq[0, h, i * 128:(i + 1) * 128] - blk)
+            assert np.all(err <= np.abs(blk) * 2.0 ** -4 + float(s[0, h, i]) * 2.0 ** -10)
+
+
+def test_smoothing_beats_unsmoothed_fp8_on_outlier_channels():
+    # the SageAttention page's claim: outlier channels in K break a plain
+    # 8-bit Q K^T; mean-centring K first makes the INT8 product accurate
+    q, k, v = make_qkv(1, 2, 2, 512, 512, 128, seed=9, dist="outlier_k")
+    qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
+    sc = 1 / math.sqrt(128)
+    O, L = oracle.attention_fp64(qb, kb, vb, True, sc)
+    Os, Ls = q8.sage8_attention_fp64(qb, kb, vb, True, sc)
+    Of, Lf = q8.fp8qk_attention_fp64(qb, kb, vb, True, sc)
+    cos = lambda a: (O * a).sum() / math.sqrt((O * O).sum() * (a * a).sum())  # noqa: E731
+    assert cos(Os) >= 0.999 > cos(Of)
+    assert np.abs(L - Ls).max() * 5 < np.abs(L - Lf).max()
