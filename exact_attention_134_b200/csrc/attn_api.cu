@@ -71,15 +71,16 @@ int device_sm_count() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// d = 96 is supported by the bf16 kernels only (allow96 = false for the 8-bit paths).
 attn_status_t check_args(const void* q, const void* k, const void* v, const void* o,
                          const void* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
-                         int causal, float scale) {
+                         int causal, float scale, bool allow96 = true) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nkv <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.0f)) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && !(allow96 && d == 96)) return ATTN_ERR_UNSUPPORTED;
   if (B > 65535 || Hq > 65535) return ATTN_ERR_UNSUPPORTED;
   // TMA global strides must stay below 2^40 bytes.
   const unsigned long long head_bytes_q = 2ull * (unsigned long long)Nq * d;
@@ -92,15 +93,16 @@ attn_status_t check_args(const void* q, const void* k, const void* v, const void
 
 // bf16 tensor [BH, N, d] as a 3-D map {d, N, BH}; box = 64 columns x 128 rows,
 // 128-byte swizzle (the layout the tcgen05 descriptors expect).
+// (d = 96: 32-column boxes with the 64-byte swizzle, three per 96-column row.)
 bool make_map(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * (cuuint64_t)d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {d == 96 ? 32u : 64u, 128, 1};
   cuuint32_t elem_strides[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
                         strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        d == 96 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -109,12 +111,12 @@ bool make_map(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
 bool make_map_packed(CUtensorMap* m, const void* ptr, int d, int H, int total) {
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)total};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * (cuuint64_t)d * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {d == 96 ? 32u : 64u, 1, 128};
   cuuint32_t elem_strides[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
                         strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        d == 96 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -300,7 +302,7 @@ namespace attn_sm100 {
 attn_status_t validate_fwd_args(const void* q, const void* k, const void* v, const void* o,
                                 const void* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
                                 int causal, float scale) {
-  return check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  return check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, false);
 }
 
 // Internal: validate arguments and run the 8-bit forward with a workspace the
@@ -310,7 +312,7 @@ attn_status_t q8_forward_with_workspace(const void* q, const void* k, const void
                                         float* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
                                         int causal, float scale, void* workspace,
                                         size_t workspace_bytes, cudaStream_t stream) {
-  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, false);
   if (s != ATTN_OK) return s;
   return run_q8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, workspace, workspace_bytes,
                 false, stream);
@@ -398,7 +400,7 @@ attn_status_t attn_q8_workspace_offsets(int B, int Hq, int Hkv, int Nq, int Nkv,
 attn_status_t attn_fwd_q8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                           int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
                           void* workspace, size_t workspace_bytes, void* stream) {
-  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, false);
   if (s != ATTN_OK) return s;
   return run_q8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, workspace,
                 workspace_bytes, false, static_cast<cudaStream_t>(stream));
@@ -408,7 +410,7 @@ attn_status_t attn_q8_prepass(const void* q, const void* k, const void* v, int B
                               int Nq, int Nkv, int d, void* workspace, size_t workspace_bytes,
                               void* stream) {
   // o / lse are not touched by the prepass; reuse the common checks with q in their place
-  attn_status_t s = check_args(q, k, v, q, q, B, Hq, Hkv, Nq, Nkv, d, 0, 1.0f);
+  attn_status_t s = check_args(q, k, v, q, q, B, Hq, Hkv, Nq, Nkv, d, 0, 1.0f, false);
   if (s != ATTN_OK) return s;
   return run_q8(q, k, v, nullptr, nullptr, B, Hq, Hkv, Nq, Nkv, d, 0, 1.0f, workspace,
                 workspace_bytes, true, static_cast<cudaStream_t>(stream));
@@ -417,7 +419,7 @@ attn_status_t attn_q8_prepass(const void* q, const void* k, const void* v, int B
 attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                            int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
                            void* workspace, size_t workspace_bytes, void* stream) {
-  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, false);
   if (s != ATTN_OK) return s;
   return run_q8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, workspace,
                 workspace_bytes, false, static_cast<cudaStream_t>(stream), true);
@@ -426,7 +428,7 @@ attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, void* o,
 attn_status_t attn_fp8_prepass(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
                                int Nq, int Nkv, int d, void* workspace, size_t workspace_bytes,
                                void* stream) {
-  attn_status_t s = check_args(q, k, v, q, q, B, Hq, Hkv, Nq, Nkv, d, 0, 1.0f);
+  attn_status_t s = check_args(q, k, v, q, q, B, Hq, Hkv, Nq, Nkv, d, 0, 1.0f, false);
   if (s != ATTN_OK) return s;
   return run_q8(q, k, v, nullptr, nullptr, B, Hq, Hkv, Nq, Nkv, d, 0, 1.0f, workspace,
                 workspace_bytes, true, static_cast<cudaStream_t>(stream), true);

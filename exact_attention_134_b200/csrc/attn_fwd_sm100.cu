@@ -43,16 +43,24 @@ constexpr int kBN = 128;  // keys per K/V tile
 constexpr int kThreads = 320;
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
-constexpr int kBoxBytes = 128 * 128;  // one TMA box: 128 rows x 64 bf16 (128 B, swizzled)
+// TMA boxes: 128 rows x kBoxCols bf16. d = 64 / 128 use 64-column boxes with
+// the 128-byte swizzle; d = 96 (192-byte rows) uses three 32-column boxes with
+// the 64-byte swizzle. The tcgen05 descriptors describe the same layouts.
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
 template <int D>
 struct FwdCfg {
   static constexpr int kTileBytes = kBM * D * 2;
-  static constexpr int kBoxes = D / 64;
-  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kBoxCols = (D == 96) ? 32 : 64;
+  static constexpr int kRowBytes = kBoxCols * 2;           // swizzle width (64 or 128 B)
+  static constexpr int kBoxBytes = kBM * kRowBytes;
+  static constexpr int kBoxes = D / kBoxCols;
+  static constexpr int kAtomBytes = 8 * kRowBytes;         // 8-row swizzle atom
+  static constexpr int kStages = (D == 128) ? 4 : (D == 96 ? 6 : 8);
+  static constexpr bool kRowStores = (D == 96);            // O stored row by row (no TMA box)
   static constexpr int kOffQ = 0;
   static constexpr int kOffRing = 2 * kTileBytes;
+  static_assert(kTileBytes % 1024 == 0, "tiles must keep the 1024-byte swizzle alignment");
   static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
   static constexpr int kBarBytes = 512;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + base alignment slack
@@ -89,9 +97,11 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint3
   constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-    const uint64_t a = smem_desc_sw128(q_smem + off, 16, 1024);
-    const uint64_t b = smem_desc_sw128(k_smem + off, 16, 1024);
+    // 16 columns (32 bytes) per MMA step: box kk / steps-per-box, then 32 B in
+    constexpr int kSteps = FwdCfg<D>::kBoxCols / 16;
+    const uint32_t off = (kk / kSteps) * FwdCfg<D>::kBoxBytes + (kk % kSteps) * 32;
+    const uint64_t a = smem_desc_sw(q_smem + off, 16, FwdCfg<D>::kAtomBytes, FwdCfg<D>::kRowBytes);
+    const uint64_t b = smem_desc_sw(k_smem + off, 16, FwdCfg<D>::kAtomBytes, FwdCfg<D>::kRowBytes);
     mma_bf16_ss(d_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
   }
 }
@@ -102,7 +112,9 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
   constexpr uint32_t idesc = idesc_bf16_f32(kBM, D, 1);
 #pragma unroll
   for (int kk = 0; kk < kBN / 16; ++kk) {
-    const uint64_t b = smem_desc_sw128(v_smem + kk * 16 * 128, kBoxBytes, 1024);
+    // V is the MN-major B operand: 16 keys = 16 rows per step; d spans boxes (LBO)
+    const uint64_t b = smem_desc_sw(v_smem + kk * 16 * FwdCfg<D>::kRowBytes, FwdCfg<D>::kBoxBytes,
+                                    FwdCfg<D>::kAtomBytes, FwdCfg<D>::kRowBytes);
     mma_bf16_ts(o_tmem, p_tmem + kk * 8, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
@@ -211,8 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(bar(BarLayout::kQFull), 2 * C::kTileBytes);
       for (int t = 0; t < 2; ++t)
         for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_load_3d(sQ + t * C::kTileBytes + bx * kBoxBytes, &tm_q, bar(BarLayout::kQFull),
-                      bx * 64, VL ? q_c1 : q_row(t), VL ? q_row(t) : bh_q);
+          tma_load_3d(sQ + t * C::kTileBytes + bx * C::kBoxBytes, &tm_q, bar(BarLayout::kQFull),
+                      bx * C::kBoxCols, VL ? q_c1 : q_row(t), VL ? q_row(t) : bh_q);
     }
     for (int j = 0; j < n_tiles && ok; ++j) {
       for (int which = 0; which < 2; ++which) {  // 0 = K_j, 1 = V_j
@@ -225,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(fb, C::kTileBytes);
           const CUtensorMap* tm = which ? &tm_v : &tm_k;
           for (int bx = 0; bx < C::kBoxes; ++bx)
-            tma_load_3d(sRing + stage * C::kTileBytes + bx * kBoxBytes, tm, fb, bx * 64,
+            tma_load_3d(sRing + stage * C::kTileBytes + bx * C::kBoxBytes, tm, fb, bx * C::kBoxCols,
                         VL ? kv_c1 : kv_row(j), VL ? kv_row(j) : bh_kv);
         }
         __syncwarp();
@@ -413,13 +425,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (ok) ok = warp_all(bounded_wait(bar(BarLayout::kOFinal), 0, abort_flag, budget));
-    if (ok && VL) {
-      // ---- epilogue (packed sequences): O = O_acc / l -> bf16 stored row by row
+    if (ok && (VL || C::kRowStores)) {
+      // ---- epilogue (packed sequences, d = 96): O = O_acc / l -> bf16 stored row by row
       tc_fence_after();
       const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
       const bool valid = row < Lq;  // q_start + row < total holds by the clamping above
-      uint4* const orow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) +
-                                                   ((size_t)(q_start + (valid ? row : 0)) * p.Hq + hq) * D);
+      const size_t orow_idx = VL ? (size_t)(q_start + (valid ? row : 0)) * p.Hq + hq
+                                 : (size_t)bh_q * p.Nq + (valid ? row : 0);
+      uint4* const orow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow_idx * D);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -437,8 +450,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (valid)  // LSE of packed sequences: [Hq, total_q]
-        p.lse[(size_t)hq * p.Nq + q_start + row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+      if (valid)  // LSE: packed sequences [Hq, total_q], dense [B, Hq, Nq]
+        p.lse[VL ? (size_t)hq * p.Nq + q_start + row : (size_t)bh_q * p.Nq + row] =
+            (m_run + log2f(l_run)) * 0.69314718055994530942f;
     } else if (ok) {
       // ---- epilogue: O = O_acc / l -> bf16 into the (now free) Q_t buffer, then TMA store
       tc_fence_after();
@@ -459,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
           v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
           v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
-          *reinterpret_cast<uint4*>(stage_ptr + bx * kBoxBytes + r * 128 + ((ch ^ (r & 7)) << 4)) = v;
+          *reinterpret_cast<uint4*>(stage_ptr + bx * C::kBoxBytes + r * 128 + ((ch ^ (r & 7)) << 4)) = v;
         }
       }
       fence_proxy_async_smem();
@@ -469,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         volatile int no_abort = 0;
         if (bounded_wait(bar(BarLayout::kEpi + t), 0, &no_abort, budget)) {
           for (int bx = 0; bx < C::kBoxes; ++bx)
-            tma_store_3d(&tm_o, sQ + t * C::kTileBytes + bx * kBoxBytes, bx * 64, q0 + t * kBM, bh_q);
+            tma_store_3d(&tm_o, sQ + t * C::kTileBytes + bx * C::kBoxBytes, bx * 64, q0 + t * kBM, bh_q);
           tma_store_commit();
           tma_store_wait_all();
         } else {
@@ -511,6 +525,9 @@ cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const 
   if (d == 128)
     return vl ? launch_fwd_d<128, true>(tq, tk, tv, to, p, stream)
               : launch_fwd_d<128, false>(tq, tk, tv, to, p, stream);
+  if (d == 96)
+    return vl ? launch_fwd_d<96, true>(tq, tk, tv, to, p, stream)
+              : launch_fwd_d<96, false>(tq, tk, tv, to, p, stream);
   return vl ? launch_fwd_d<64, true>(tq, tk, tv, to, p, stream)
             : launch_fwd_d<64, false>(tq, tk, tv, to, p, stream);
 }

@@ -79,6 +79,12 @@ SMALL = [
     (2, 4, 1, 512, 64, 64, False),
     (1, 2, 2, 640, 1900, 128, False),
     (1, 16, 2, 1024, 1024, 128, True),
+    # head dim 96: three 32-column boxes per row
+    (1, 2, 2, 256, 256, 96, False),
+    (1, 4, 2, 300, 300, 96, True),
+    (2, 8, 1, 513, 513, 96, True),
+    (1, 2, 2, 100, 777, 96, False),
+    (1, 2, 2, 200, 650, 96, True),
 ]
 
 

@@ -83,6 +83,7 @@ VARLEN = [
     ([64, 200, 513], [1000, 200, 700], 8, 2, 128, True),     # prefill with a cache
     ([300, 50, 5], [100, 0, 5], 2, 2, 128, True),            # Lq > Lk, an empty key set
     ([700, 0, 33], [700, 40, 33], 4, 4, 64, True),           # an empty query sequence
+    ([129, 64, 300], [129, 500, 300], 4, 2, 96, True),       # head dim 96
 ]
 
 
