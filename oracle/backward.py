@@ -1,0 +1,53 @@
+"""Attention backward in fp64 from the derivative of the definition (test
+infrastructure).
+
+The glossary page "FlashAttention" (aisaas-seo) says the backward pass
+recomputes the few cheap intermediates instead of storing them; the gradients
+themselves follow from differentiating O = softmax(scale * Q K^T) V (the
+definition on "FlashAttention (TR)", "Standart Attention Mekanizmasının
+Sorunları"). For one (batch, head), with P the softmax probabilities:
+
+    dV  = P^T dO
+    dP  = dO V^T
+    dS  = P * (dP - rowsum(P * dP))        (softmax Jacobian, row by row)
+    dQ  = scale * dS K
+    dK  = scale * dS^T Q
+
+GQA: a kv head's dK and dV are the sums over the query heads of its group.
+Masked positions have P = 0 and hence dS = 0. Everything in float64 on the
+exact bf16 inputs.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .attention import _kv_head, score_matrix_fp64, widen_bf16
+
+
+def attention_bwd_fp64(q_bits, k_bits, v_bits, do_bits, causal: bool, scale: float):
+    """q_bits, do_bits: uint16 [B, Hq, Nq, d]; k_bits, v_bits: uint16 [B, Hkv, Nkv, d].
+    Returns (dQ [B, Hq, Nq, d], dK [B, Hkv, Nkv, d], dV [B, Hkv, Nkv, d]) float64."""
+    B, Hq, Nq, d = q_bits.shape
+    Hkv, Nkv = k_bits.shape[1], k_bits.shape[2]
+    dQ = np.zeros((B, Hq, Nq, d))
+    dK = np.zeros((B, Hkv, Nkv, d))
+    dV = np.zeros((B, Hkv, Nkv, d))
+    for b in range(B):
+        for h in range(Hq):
+            hk = _kv_head(h, Hq, Hkv)
+            q = widen_bf16(q_bits[b, h])
+            k = widen_bf16(k_bits[b, hk])
+            v = widen_bf16(v_bits[b, hk])
+            do = widen_bf16(do_bits[b, h])
+            S = score_matrix_fp64(q, k, scale, causal)
+            m = S.max(axis=1)
+            empty = np.isinf(m)
+            E = np.exp(S - np.where(empty, 0.0, m)[:, None])
+            l = E.sum(axis=1)
+            P = np.where(empty[:, None], 0.0, E / np.where(empty, 1.0, l)[:, None])
+            dV[b, hk] += P.T @ do
+            dP = do @ v.T
+            dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+            dQ[b, h] = scale * (dS @ k)
+            dK[b, hk] += scale * (dS.T @ q)
+    return dQ, dK, dV

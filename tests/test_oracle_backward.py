@@ -1,0 +1,77 @@
+"""Pins for the fp64 backward oracle (CPU only): torch autograd in float64 on
+the same definition (a library special case), central finite differences of
+a scalar loss (brute force), and the identity rowsum(P * dP) = rowsum(dO * O)
+the kernels rely on."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synthetic import bf16_bits, make_qkv
+
+
+def _inputs(B, Hq, Hkv, Nq, Nkv, d, seed):
+    q, k, v = make_qkv(B, Hq, Hkv, Nq, Nkv, d, seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    do = torch.randn((B, Hq, Nq, d), generator=g).to(torch.bfloat16)
+    return bf16_bits(q), bf16_bits(k), bf16_bits(v), bf16_bits(do)
+
+
+def _autograd(qb, kb, vb, dob, causal, scale):
+    q, k, v, do = (torch.from_numpy(oracle.widen_bf16(x)).requires_grad_(True) for x in (qb, kb, vb, dob))
+    g = q.shape[1] // k.shape[1]
+    Nq, Nkv = q.shape[2], k.shape[2]
+    mask = None
+    if causal:
+        mask = torch.arange(Nkv)[None, :] <= torch.arange(Nq)[:, None] + (Nkv - Nq)
+    o = torch.nn.functional.scaled_dot_product_attention(
+        q, k.repeat_interleave(g, dim=1), v.repeat_interleave(g, dim=1), attn_mask=mask, scale=scale)
+    o.backward(do.detach())
+    return q.grad.numpy(), k.grad.numpy(), v.grad.numpy()
+
+
+@pytest.mark.parametrize("shape,causal", [
+    ((1, 2, 2, 33, 33, 16), False), ((2, 4, 2, 40, 40, 8), True), ((1, 4, 1, 17, 60, 16), True),
+    ((1, 2, 2, 64, 20, 8), False),
+])
+def test_backward_matches_torch_autograd(shape, causal):
+    qb, kb, vb, dob = _inputs(*shape, seed=sum(shape))
+    scale = 1 / math.sqrt(shape[-1])
+    dQ, dK, dV = oracle.attention_bwd_fp64(qb, kb, vb, dob, causal, scale)
+    rq, rk, rv = _autograd(qb, kb, vb, dob, causal, scale)
+    for a, r in ((dQ, rq), (dK, rk), (dV, rv)):
+        assert np.max(np.abs(a - r)) < 1e-11
+
+
+def test_backward_finite_differences():
+    qb, kb, vb, dob = _inputs(1, 2, 1, 6, 7, 4, seed=5)
+    scale = 0.4
+    dQ, dK, dV = oracle.attention_bwd_fp64(qb, kb, vb, dob, True, scale)
+    q, k, v, do = (oracle.widen_bf16(x) for x in (qb, kb, vb, dob))
+
+    def loss(q_, k_, v_):
+        O, _ = oracle.attention_f64(q_, k_, v_, True, scale)
+        return float((O * do).sum())
+    eps = 1e-6
+    for x, g in ((q, dQ), (k, dK), (v, dV)):
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [xp if x is a else a for a in (q, k, v)]
+            args_m = [xm if x is a else a for a in (q, k, v)]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - g[idx]) < 1e-7
+
+
+def test_delta_identity():
+    qb, kb, vb, dob = _inputs(1, 2, 2, 50, 50, 16, seed=9)
+    O, _, P = oracle.attention_fp64(qb, kb, vb, True, 0.25, return_p=True)
+    do = oracle.widen_bf16(dob)
+    v = oracle.widen_bf16(vb)
+    dP = np.einsum("bhid,bhjd->bhij", do, v)
+    assert np.max(np.abs((P * dP).sum(-1) - (do * O).sum(-1))) < 1e-12
