@@ -1,4 +1,4 @@
-"""B200 (sm_100a) fused exact attention forward — Python binding.
+"""B200 (sm_100a) fused exact attention (forward and backward) — Python binding.
 
 A thin ctypes layer over the C ABI in ``include/attn.h`` (the in-tree library
 ``libattn_b200.so``). It only marshals arguments: it checks dtypes, devices and
@@ -8,6 +8,7 @@ kernels; there is no other implementation to fall back to — if the library is
 missing or cannot run, the call raises.
 
     o, lse = attn_fwd(q, k, v, causal=True)          # bf16 [B,H,N,d] on cuda
+    dq, dk, dv = attn_bwd(q, k, v, o, lse, do, causal=True)
 """
 from __future__ import annotations
 
@@ -51,6 +52,8 @@ _SIGNATURES = {
     "attn_fwd_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp, _sz, _vp]),
     "attn_fp8_prepass": (_c_int, [_vp, _vp, _vp] + [_c_int] * 6 + [_vp, _sz, _vp]),
     "attn_q8_workspace_offsets": (_c_int, [_c_int] * 6 + [ctypes.POINTER(_sz)]),
+    "attn_bwd_workspace_size": (_sz, [_c_int] * 6),
+    "attn_bwd": (_c_int, [_vp] * 9 + [_c_int] * 7 + [_c_float, _vp, _sz, _vp]),
     "attn_get_status": (_c_int, [_vp]),
     "attn_get_status_ex": (_c_int, [_vp, ctypes.POINTER(_c_int)]),
     "attn_set_timeout_ms": (_c_int, [_c_int]),
@@ -160,6 +163,46 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, caus
                                int(bool(causal)), float(scale), _stream_handle(q.device))
     _check(st, "attn_fwd_varlen")
     return out, lse
+
+
+def bwd_workspace_size(B, Hq, Hkv, Nq, Nkv, d) -> int:
+    return int(lib().attn_bwd_workspace_size(B, Hq, Hkv, Nq, Nkv, d))
+
+
+def attn_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
+             workspace=None, dq=None, dk=None, dv=None):
+    """Gradients of attn_fwd on the GPU.
+
+    q, o, dout: bf16 cuda [B, Hq, Nq, d]; k, v: bf16 cuda [B, Hkv, Nkv, d];
+    lse: fp32 cuda [B, Hq, Nq] (the forward's). Returns (dq, dk, dv) in the
+    layouts of q, k, v. `workspace` (uint8 cuda, >= bwd_workspace_size bytes)
+    is allocated when not given.
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    B, Hq, Hkv, Nq, Nkv, d = _shape_args(q, k, v)
+    if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("o and dout must have the shape of q")
+    if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous() or \
+            tuple(lse.shape) != (B, Hq, Nq):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, Hq, Nq]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = bwd_workspace_size(B, Hq, Hkv, Nq, Nkv, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = lib().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                        dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                        B, Hq, Hkv, Nq, Nkv, d, int(bool(causal)), float(scale),
+                        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                        _stream_handle(q.device))
+    _check(st, "attn_bwd")
+    return dq, dk, dv
 
 
 def q8_workspace_size(B, Hq, Hkv, Nq, Nkv, d) -> int:

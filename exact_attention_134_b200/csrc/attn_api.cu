@@ -294,6 +294,73 @@ HostLayout host_layout(int B, int Hq, int Hkv, int Nq, int Nkv, int d) {
   return L;
 }
 
+// Backward workspace: fp32 dQ accumulator [B*Hq, nq_pad, d], then LSE*log2(e)
+// and D, each [B*Hq, nq_pad] fp32; regions 256-byte aligned.
+struct BwdLayout {
+  size_t acc, lse2, dvec, total;
+};
+
+BwdLayout bwd_layout(int B, int Hq, int Nq, int d) {
+  const size_t rows = (size_t)B * Hq * (size_t)((Nq + 127) / 128 * 128);
+  BwdLayout L;
+  L.acc = 0;
+  L.lse2 = round_up(L.acc + 4 * rows * d, 256);
+  L.dvec = round_up(L.lse2 + 4 * rows, 256);
+  L.total = round_up(L.dvec + 4 * rows, 256);
+  return L;
+}
+
+attn_status_t run_bwd(const void* q, const void* k, const void* v, const void* o,
+                      const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                      int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
+                      void* workspace, cudaStream_t stream) {
+  int* status = device_status_ptr();
+  if (!status) return ATTN_ERR_CUDA;
+  const BwdLayout W = bwd_layout(B, Hq, Nq, d);
+  char* w = static_cast<char*>(workspace);
+  attn_sm100::BwdLaunch L;
+  std::memset(static_cast<void*>(&L), 0, sizeof(L));
+  if (!make_map(&L.tq, q, d, Nq, (long long)B * Hq) || !make_map(&L.tk, k, d, Nkv, (long long)B * Hkv) ||
+      !make_map(&L.tv, v, d, Nkv, (long long)B * Hkv) ||
+      !make_map(&L.tdo, dout, d, Nq, (long long)B * Hq))
+    return ATTN_ERR_CUDA;
+  const int nq_pad = (Nq + 127) / 128 * 128;
+  float* acc = reinterpret_cast<float*>(w + W.acc);
+  float* lse2 = reinterpret_cast<float*>(w + W.lse2);
+  float* dvec = reinterpret_cast<float*>(w + W.dvec);
+  L.B = B;
+  L.pre.o = o;
+  L.pre.dout = dout;
+  L.pre.lse = lse;
+  L.pre.dvec = dvec;
+  L.pre.lse2 = lse2;
+  L.pre.dq_acc = acc;
+  L.pre.Nq = Nq;
+  L.pre.nq_pad = nq_pad;
+  attn_sm100::BwdParams& p = L.main;
+  p.dk = dk;
+  p.dv = dv;
+  p.dq_acc = acc;
+  p.lse2 = lse2;
+  p.dvec = dvec;
+  p.status = status;
+  p.Nq = Nq;
+  p.Nkv = Nkv;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.causal = causal;
+  p.nq_pad = nq_pad;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = (unsigned long long)g_timeout_ns.load();
+  L.post.dq_acc = acc;
+  L.post.dq = dq;
+  L.post.Nq = Nq;
+  L.post.nq_pad = nq_pad;
+  L.post.scale = scale;
+  return cuda_status(attn_sm100::launch_bwd(L, d, stream));
+}
+
 }  // namespace
 
 namespace attn_sm100 {
@@ -432,6 +499,27 @@ attn_status_t attn_fp8_prepass(const void* q, const void* k, const void* v, int 
   if (s != ATTN_OK) return s;
   return run_q8(q, k, v, nullptr, nullptr, B, Hq, Hkv, Nq, Nkv, d, 0, 1.0f, workspace,
                 workspace_bytes, true, static_cast<cudaStream_t>(stream), true);
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nkv, int d) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nkv <= 0 || d <= 0) return 0;
+  return bwd_layout(B, Hq, Nq, d).total;
+}
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                       const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                       int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, false);
+  if (s != ATTN_OK) return s;
+  if (!dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+  if ((long long)B * Hq > 65535) return ATTN_ERR_UNSUPPORTED;  // grid y of the row kernels
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return ATTN_ERR_ALIGNMENT;
+  if (!workspace || !aligned16(workspace) ||
+      workspace_bytes < bwd_layout(B, Hq, Nq, d).total)
+    return ATTN_ERR_WORKSPACE;
+  return run_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nkv, d, causal, scale,
+                 workspace, static_cast<cudaStream_t>(stream));
 }
 
 attn_status_t attn_get_status_ex(void* stream, int* where) {

@@ -63,6 +63,49 @@ struct Q8Launch {
 
 cudaError_t launch_q8(const Q8Launch& L, int d, cudaStream_t stream);
 
+// Backward main kernel parameters (tensor maps of Q, K, V, dO passed separately).
+struct BwdParams {
+  void* dk;                       // bf16 [B, Hkv, Nkv, d]
+  void* dv;                       // bf16 [B, Hkv, Nkv, d]
+  float* dq_acc;                  // fp32 [B*Hq][nq_pad/32][d/4][32][4]
+  const float* lse2;              // fp32 [B*Hq][nq_pad]  LSE * log2(e), +inf where P must be 0
+  const float* dvec;              // fp32 [B*Hq][nq_pad]  D_i = sum_c dO_ic O_ic
+  int* status;
+  int Nq, Nkv, Hq, Hkv;
+  int causal;
+  int nq_pad;                     // Nq rounded up to 128
+  float scale;
+  float scale_log2;
+  unsigned long long timeout_ns;
+};
+
+struct BwdPreParams {
+  const void* o;                  // bf16 [B, Hq, Nq, d]
+  const void* dout;               // bf16 [B, Hq, Nq, d]
+  const float* lse;               // fp32 [B, Hq, Nq]
+  float* dvec;
+  float* lse2;
+  float* dq_acc;
+  int Nq, nq_pad;
+};
+
+struct BwdPostParams {
+  const float* dq_acc;
+  void* dq;                       // bf16 [B, Hq, Nq, d]
+  int Nq, nq_pad;
+  float scale;
+};
+
+struct BwdLaunch {
+  CUtensorMap tq, tk, tv, tdo;
+  BwdParams main;
+  BwdPreParams pre;
+  BwdPostParams post;
+  int B;
+};
+
+cudaError_t launch_bwd(const BwdLaunch& L, int d, cudaStream_t stream);
+
 attn_status_t validate_fwd_args(const void* q, const void* k, const void* v, const void* o,
                                 const void* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
                                 int causal, float scale);

@@ -206,6 +206,37 @@ ATTN_API attn_status_t attn_q8_workspace_offsets(int B, int Hq, int Hkv, int Nq,
                                                  size_t* offsets);
 
 /*
+ * attn_bwd — gradients of attn_fwd: given dO = dLoss/dO, writes
+ *     dQ = scale * dS K,   dK = scale * dS^T Q,   dV = P^T dO,
+ *     dS = P * (dO V^T - D),   D_i = sum_c dO_ic O_ic,
+ * with P = exp(scale * Q K^T - LSE) recomputed block by block from the LSE the
+ * forward wrote (the glossary page "FlashAttention", aisaas-seo: the backward
+ * recomputes a few cheap quantities instead of storing them); no N x N matrix
+ * is stored. The formulas are the derivative of the definition on
+ * "FlashAttention (TR)" ("Standart Attention Mekanizmasının Sorunları").
+ *   q, k, v        bf16 inputs of the forward, layouts as attn_fwd
+ *   o, lse         the forward's outputs (bf16 [B,Hq,Nq,d], fp32 [B,Hq,Nq])
+ *   dout           bf16 [B, Hq, Nq, d]
+ *   dq             bf16 [B, Hq, Nq, d]   (written)
+ *   dk, dv         bf16 [B, Hkv, Nkv, d] (written; with GQA the sum over the
+ *                  query heads of each group)
+ *   causal, scale  as passed to the forward (bottom-right causal alignment)
+ *   workspace      device scratch of attn_bwd_workspace_size() bytes, 16-byte
+ *                  aligned, owned by the caller; holds the fp32 dQ
+ *                  accumulator, D and LSE * log2(e); needs no initial value
+ * d must be 64 or 128 (96: ATTN_ERR_UNSUPPORTED), B * Hq <= 65535. The dQ accumulation adds
+ * fp32 partial sums with atomics, so dQ may differ in the last bits between
+ * runs; dK and dV are deterministic. Errors as attn_fwd, plus
+ * ATTN_ERR_WORKSPACE for a missing, misaligned or short workspace.
+ */
+ATTN_API size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nkv, int d);
+ATTN_API attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                int B, int Hq, int Hkv, int Nq, int Nkv, int d, int causal,
+                                float scale, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/*
  * attn_get_status — synchronises `stream`, returns and clears the device
  * status word (ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel gave up on a pipeline
  * wait since the last call). Returns ATTN_ERR_CUDA if synchronisation fails.

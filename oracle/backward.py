@@ -51,3 +51,47 @@ def attention_bwd_fp64(q_bits, k_bits, v_bits, do_bits, causal: bool, scale: flo
             dQ[b, h] = scale * (dS @ k)
             dK[b, hk] += scale * (dS.T @ q)
     return dQ, dK, dV
+
+
+def attention_bwd_head_blocks(q, k, v, do, causal: bool, scale: float, block_rows: int = 2048):
+    """One (batch, query head) of the same computation on float64 arrays
+    q, do [Nq, d] and k, v [Nkv, d], walked over blocks of query rows so that
+    long sequences fit in memory. Every row of a block is complete (all of its
+    keys), so each yielded quantity is exact for its rows:
+
+        dict(i0, i1, S (scaled, masked -inf), P, O, LSE, D, dP, dS)
+
+    The gradients of the head are then dQ[i0:i1] = scale * dS K and the sums
+    over blocks of scale * dS^T Q[i0:i1] (dK) and P^T dO[i0:i1] (dV)."""
+    Nq, Nkv = q.shape[0], k.shape[0]
+    off = Nkv - Nq
+    for i0 in range(0, Nq, block_rows):
+        i1 = min(Nq, i0 + block_rows)
+        S = (q[i0:i1] @ k.T) * scale
+        if causal:
+            rows = np.arange(i0, i1)[:, None]
+            S = np.where(np.arange(Nkv)[None, :] <= rows + off, S, -np.inf)
+        m = S.max(axis=1)
+        empty = np.isinf(m)
+        E = np.exp(S - np.where(empty, 0.0, m)[:, None])
+        l = E.sum(axis=1)
+        P = np.where(empty[:, None], 0.0, E / np.where(empty, 1.0, l)[:, None])
+        lse = np.where(empty, -np.inf, m + np.log(np.where(empty, 1.0, l)))
+        O = P @ v
+        D = (do[i0:i1] * O).sum(axis=1)
+        dP = do[i0:i1] @ v.T
+        dS = P * (dP - D[:, None])
+        yield dict(i0=i0, i1=i1, S=S, P=P, O=O, LSE=lse, D=D, dP=dP, dS=dS)
+
+
+def attention_bwd_head(q, k, v, do, causal: bool, scale: float, block_rows: int = 2048):
+    """dQ [Nq, d], dK, dV [Nkv, d] of one head from attention_bwd_head_blocks."""
+    dQ = np.zeros_like(q)
+    dK = np.zeros_like(k)
+    dV = np.zeros_like(v)
+    for blk in attention_bwd_head_blocks(q, k, v, do, causal, scale, block_rows):
+        i0, i1 = blk["i0"], blk["i1"]
+        dQ[i0:i1] = scale * (blk["dS"] @ k)
+        dK += scale * (blk["dS"].T @ q[i0:i1])
+        dV += blk["P"].T @ do[i0:i1]
+    return dQ, dK, dV

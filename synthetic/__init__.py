@@ -6,7 +6,7 @@ and rounds them to bf16. Every workload below stands in for the model-level
 workloads the FlashAttention / SageAttention pages measure on (BERT, GPT-2,
 Long-Range Arena, video diffusion), which are not available here.
 
-Recipe (same for every workload):
+Recipe (same for every workload; the backward's dO: see ``make_dout``):
   * ``torch.Generator('cpu').manual_seed(seed)``;
   * fp32 ``randn`` draws in the order Q, K, V, then any extras;
   * the "outlier K" distribution adds a per-(kv head, channel) offset b that is
@@ -105,6 +105,13 @@ def make_qkv(B: int, Hq: int, Hkv: int, Nq: int, Nkv: int, d: int, seed: int,
 
 def make_workload(w: Workload):
     return make_qkv(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.seed, w.dist)
+
+
+def make_dout(B: int, Hq: int, Nq: int, d: int, seed: int) -> torch.Tensor:
+    """The upstream gradient dO for a backward pass: fp32 ``randn`` from its
+    own generator seeded with ``seed + 500``, rounded to bf16 [B, Hq, Nq, d]."""
+    g = torch.Generator("cpu").manual_seed(seed + 500)
+    return _bf16(torch.randn((B, Hq, Nq, d), generator=g, dtype=torch.float32))
 
 
 def sample_rows(w: Workload, n_rows: int | None = None, seed_offset: int = 77):

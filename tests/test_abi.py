@@ -108,3 +108,20 @@ def test_varlen_entry_validation(lib):
     assert call(scale=float("nan")) == 1 and call(causal=3) == 1
     assert call(d=80) == 2 and call(n=70000) == 2
     assert call(q=P + 2) == 3 and call(cq=P + 2) == 3
+
+
+def test_bwd_entry_validation(lib):
+    need = lib.attn_bwd_workspace_size(2, 4, 2, 300, 500, 128)
+    # fp32 dQ accumulator over 384 padded rows, then LSE_2 and D, 256-byte aligned
+    rows = 2 * 4 * 384
+    assert need >= 4 * rows * 128 + 8 * rows and need % 256 == 0
+    assert lib.attn_bwd_workspace_size(0, 4, 2, 300, 500, 128) == 0
+
+    def call(dq=P, ws=P, nbytes=need, d=128, Hq=4, B=2, causal=1, scale=0.1, dout=P):
+        return lib.attn_bwd(P, P, P, P, P, dout, dq, P, P, B, Hq, 2, 300, 500, d, causal, scale,
+                            ws, nbytes, None)
+    assert call(dq=None) == 1 and call(dout=None) == 1 and call(Hq=3) == 1
+    assert call(causal=2) == 1 and call(scale=-1.0) == 1
+    assert call(d=96) == 2 and call(B=40000, Hq=4) == 2
+    assert call(dq=P + 4) == 3
+    assert call(ws=None) == 6 and call(ws=P + 8) == 6 and call(nbytes=need - 1) == 6

@@ -75,3 +75,26 @@ def test_delta_identity():
     v = oracle.widen_bf16(vb)
     dP = np.einsum("bhid,bhjd->bhij", do, v)
     assert np.max(np.abs((P * dP).sum(-1) - (do * O).sum(-1))) < 1e-12
+
+
+@pytest.mark.parametrize("block_rows", [7, 16, 1000])
+def test_row_blocked_head_matches_whole_matrix(block_rows):
+    qb, kb, vb, dob = _inputs(1, 2, 1, 45, 60, 16, seed=12)
+    scale = 0.3
+    dQ, dK, dV = oracle.attention_bwd_fp64(qb, kb, vb, dob, True, scale)
+    w = oracle.widen_bf16
+    gK = np.zeros_like(dK[0, 0])
+    gV = np.zeros_like(dV[0, 0])
+    for h in range(2):
+        q, do = w(qb[0, h]), w(dob[0, h])
+        k, v = w(kb[0, 0]), w(vb[0, 0])
+        hq, hk, hv = oracle.backward.attention_bwd_head(q, k, v, do, True, scale, block_rows)
+        assert np.max(np.abs(hq - dQ[0, h])) < 1e-13
+        gK += hk
+        gV += hv
+        # the blocks' O and LSE are the forward's
+        O, L = oracle.attention_f64(q[None, None], k[None, None], v[None, None], True, scale)
+        for blk in oracle.backward.attention_bwd_head_blocks(q, k, v, do, True, scale, block_rows):
+            assert np.max(np.abs(blk["O"] - O[0, 0, blk["i0"]:blk["i1"]])) < 1e-13
+            assert np.max(np.abs(blk["LSE"] - L[0, 0, blk["i0"]:blk["i1"]])) < 1e-13
+    assert np.max(np.abs(gK - dK[0, 0])) < 1e-13 and np.max(np.abs(gV - dV[0, 0])) < 1e-13
