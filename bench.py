@@ -29,7 +29,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synthetic import (VARLEN_WORKLOADS, WORKLOADS, Workload, bf16_bits, make_qkv,  # noqa: E402
+from synthetic import (VARLEN_WORKLOADS, WORKLOADS, Workload, bf16_bits, make_dout, make_qkv,  # noqa: E402
                        make_varlen)
 
 HEADLINE = "outlier_8k_causal"
@@ -293,6 +293,40 @@ def bench_varlen(name: str, steps: int, warmup: int, world: int, lib_mod):
             "l2": "inputs_larger_than_l2"}
 
 
+BWD_WORKLOADS = ["outlier_8k_causal", "outlier_8k_full", "gqa_32k_d128"]
+
+
+def bench_bwd(w: Workload, steps: int, warmup: int, world: int, rank: int, lib_mod, peak: float):
+    """Backward (attn_bwd: preprocess, main and dQ-conversion kernels) after
+    one forward that provides O and LSE; inputs larger than L2. FLOPs counted
+    as 2.5 x the forward's (five N x N x d products instead of two)."""
+    import torch
+    wr = rank_workload(w, rank)
+    q, k, v = make_qkv(wr.B, wr.Hq, wr.Hkv, wr.Nq, wr.Nkv, wr.d, wr.seed, wr.dist)
+    do = make_dout(wr.B, wr.Hq, wr.Nq, wr.d, wr.seed)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, lse = lib_mod.attn_fwd(qd, kd, vd, causal=w.causal)
+    ws = torch.empty(lib_mod.bwd_workspace_size(wr.B, wr.Hq, wr.Hkv, wr.Nq, wr.Nkv, wr.d),
+                     dtype=torch.uint8, device="cuda")
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+
+    def step():
+        lib_mod.attn_bwd(qd, kd, vd, o, lse, dod, causal=w.causal, workspace=ws, dq=dq, dk=dk, dv=dv)
+
+    _barrier(world)
+    times = time_device(step, steps, max(warmup, 3))
+    _barrier(world)
+    st, where = lib_mod.get_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} at {where:#x}")
+    ms = _max_over_ranks(statistics.mean(times), world)
+    tf = world * 2.5 * w.flops / (ms * 1e-3) / 1e12
+    return {"tflops": round(tf, 1), "ms_per_step": round(ms, 4),
+            "frac_of_bf16_peak": round(tf / world / peak, 4),
+            "flops": "2.5 x forward (five N x N x d products)", "launches_per_step": 3,
+            "l2": "inputs_larger_than_l2"}
+
+
 def bench_e2e(w: Workload, steps: int, warmup: int, world: int, rank: int, lib_mod):
     """Same metric through the host-buffer entry point: every step copies the
     step's inputs from pinned host memory and reads O and LSE back."""
@@ -387,6 +421,10 @@ def run_ours(args):
         extras["varlen_prefill_mixed"] = bench_varlen("varlen_prefill_mixed", max(3, args.steps // 2),
                                                       3, world, attn)
         torch.cuda.empty_cache()
+        for name in BWD_WORKLOADS:
+            extras["backward_" + name] = bench_bwd(WORKLOADS[name], max(3, args.steps // 2), 3, world,
+                                                   rank, attn, peaks["bf16"])
+            torch.cuda.empty_cache()
         wq = WORKLOADS["q8_8k_outlier"]
         full_ms, pre_ms = bench_q8(wq, max(3, args.steps // 2), 3, world, rank, attn)
         fp8_peak = 2.0 * peaks["bf16"]
@@ -445,6 +483,29 @@ def run_ours(args):
         print(json.dumps(out), flush=True)
 
 
+def run_bwd_only(args):
+    """Only the backward of one workload (for timing and profiling it alone):
+    one JSON line with its device-timed TFLOP/s."""
+    import exact_attention_134_b200 as attn
+    world, rank, _ = _dist_setup()
+    peaks = _peaks()
+    w = WORKLOADS[args.workload]
+    attn.lib()
+    r = bench_bwd(w, args.steps, args.warmup, world, rank, attn, peaks["bf16"])
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps({"metric": "attention backward throughput (dQ, dK, dV)", "value": r["tflops"],
+                          "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                          "warmup": max(args.warmup, 3), "ms_per_step": r["ms_per_step"],
+                          "higher_is_better": True, "scaling": "weak", "dtype": "bf16",
+                          "data": "synthetic", "config": {"workload": w.name, "direction": "bwd",
+                                                          "l2": r["l2"], "flops": r["flops"]},
+                          "frac_of_bf16_peak": r["frac_of_bf16_peak"]}), flush=True)
+
+
 def run_reference(args):
     """The oracle on host cores, timed per step over a bounded sample."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -487,9 +548,13 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--kernel-only", action="store_true",
                     help="only the device-timed leg (for profiling runs): no e2e, CPU or extra legs")
+    ap.add_argument("--direction", default="fwd", choices=["fwd", "bwd"],
+                    help="bwd: time only the backward of --workload (one JSON line)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.direction == "bwd":
+        run_bwd_only(args)
     else:
         run_ours(args)
 

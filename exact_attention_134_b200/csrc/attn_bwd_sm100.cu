@@ -16,8 +16,9 @@
 // (TMEM), and streams the query blocks of every query head of its group past
 // them. Three kernels:
 //   attn_bwd_pre   D = rowsum(dO * O), LSE in log2 units, zeroed dQ accumulator
-//   attn_bwd_main  everything else; dQ partial sums are added into an fp32
-//                  accumulator with vector atomics (each key block contributes)
+//   attn_bwd_main  everything else; each key block's dQ partial sums are
+//                  staged in shared memory and added into an fp32 accumulator
+//                  by the TMA unit (cp.reduce.async.bulk .add.f32)
 //   attn_bwd_post  dQ = bf16(scale * accumulator)
 //
 // Main kernel, per iteration (one 128-row query block of one query head):
@@ -31,8 +32,9 @@
 //   dQ_j = dS K                 (SS MMA, A = the dS tile read MN-major)
 // Roles (384 threads, three warpgroups):
 //   warps 0-3  P and dS (thread = key row = TMEM lane), then the dK epilogue
-//   warps 4-7  dQ drain (thread = query row): TMEM -> registers -> atomics,
-//              then the dV epilogue
+//   warps 4-7  dQ drain (thread = query row): TMEM -> registers -> the dO
+//              buffer of the finished query block, 16 KB at a time -> bulk
+//              reduce-add into the accumulator; then the dV epilogue
 //   warp  8    MMA issuer
 //   warp  9    TMA producer (K, V once; Q, dO, LSE_2, D per query block)
 //   warps 10-11 idle (they complete the third warpgroup, which the register
@@ -45,6 +47,12 @@
 // tcgen05 MMAs from one thread execute in issue order, so S(it+1) overwrites
 // P^T(it) only after dV(it) read it, and dQ(it) overwrites dS^T(it) only after
 // dK(it) read it; dP(it+1) waits until the dQ drain has read dQ(it).
+// Each query-block stage has two halves with their own barriers: Q and LSE_2
+// are released when dK(it) completes, dO and D only when the dQ drain's bulk
+// reductions have read the dO buffer (it doubles as their staging area).
+// Measured on B200: vector atomics (red.global.add.v4.f32) from registers for
+// the same 64 KB per iteration stalled the tensor core's shared-memory
+// operand reads while they drained; the bulk reduce does not.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -80,7 +88,8 @@ struct BwdCfg {
   // the tiles to the 1024-byte swizzle atom; the kernel checks the base it got
   static constexpr int kSlack = (kBytes + 1024 <= kMaxSmem) ? 1024 : (kMaxSmem - kBytes);
   static constexpr int kSmemBytes = kBytes + kSlack;
-  static constexpr int kStageBytes = 2 * kTileBytes + 2 * kBQ * 4;  // TMA bytes per query block
+  static constexpr int kHalfBytes = kTileBytes + kBQ * 4;  // TMA bytes of Q + LSE_2 (or dO + D)
+  static constexpr int kStageBufs = kTileBytes / 16384;      // 16 KB dQ staging buffers in a dO tile
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
   static_assert(kBytes <= kMaxSmem, "shared memory layout too large");
 };
@@ -88,8 +97,8 @@ struct BwdCfg {
 // Barrier slots (8 bytes each).
 struct Bars {
   static constexpr int kKV = 0;
-  static constexpr int kFull = 1;    // [2]
-  static constexpr int kEmpty = 3;   // [2]
+  static constexpr int kFull = 1;    // [2] Q + LSE_2 of stage s landed
+  static constexpr int kEmpty = 3;   // [2] Q + LSE_2 of stage s released (dK done)
   static constexpr int kS = 5;       // S^T(it) in TMEM
   static constexpr int kDP = 6;      // dP^T(it) in TMEM
   static constexpr int kP = 7;       // P^T(it) written (128 arrivals)
@@ -98,8 +107,10 @@ struct Bars {
   static constexpr int kDQFree = 10; // dQ(it) read out of TMEM (128 arrivals)
   static constexpr int kAcc = 11;    // dK, dV final
   static constexpr int kDrain = 12;
-  static constexpr int kTmemSlotByte = 8 * 13;
-  static constexpr int kAbortByte = 8 * 13 + 4;
+  static constexpr int kFullDO = 13;  // [2] dO + D of stage s landed
+  static constexpr int kEmptyDO = 15; // [2] dO buffer of stage s released (dQ staged out)
+  static constexpr int kTmemSlotByte = 8 * 17;
+  static constexpr int kAbortByte = 8 * 17 + 4;
 };
 
 __device__ __forceinline__ void flag_abort(volatile int* abort_flag, int* status, int where) {
@@ -232,6 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(Bars::kFull + s), 1);
       mbar_init(bar(Bars::kEmpty + s), 1);
+      mbar_init(bar(Bars::kFullDO + s), 1);
+      mbar_init(bar(Bars::kEmptyDO + s), 1);
     }
     mbar_init(bar(Bars::kS), 1);
     mbar_init(bar(Bars::kDP), 1);
@@ -275,33 +288,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sV + bx * C::kBoxBytes, &tm_v, bar(Bars::kKV), bx * 64, k0, bh_kv);
       }
     }
-    for (; it < n_iter && ok; ++it) {
+    int half = 0;  // 0: Q + LSE_2 of query block it; 1: its dO + D
+    for (; it < n_iter && ok; half ^= 1, it += half ^ 1) {
       const int s = it & 1;
-      ok = warp_all(bounded_wait(bar(Bars::kEmpty + s), ((it >> 1) & 1) ^ 1, abort_flag, budget));
+      ok = warp_all(bounded_wait(bar((half ? Bars::kEmptyDO : Bars::kEmpty) + s),
+                                 ((it >> 1) & 1) ^ 1, abort_flag, budget));
       if (!ok) break;
       if (lane == 0) {
         const int q0 = q_block(it) * kBQ;
         const int bh_q = b * p.Hq + q_head(it);
-        const uint32_t fb = bar(Bars::kFull + s);
-        mbar_arrive_expect_tx(fb, C::kStageBytes);
-        for (int bx = 0; bx < C::kBoxes; ++bx) {
-          tma_load_3d(sQ(s) + bx * C::kBoxBytes, &tm_q, fb, bx * 64, q0, bh_q);
-          tma_load_3d(sDO(s) + bx * C::kBoxBytes, &tm_do, fb, bx * 64, q0, bh_q);
-        }
+        const uint32_t fb = bar((half ? Bars::kFullDO : Bars::kFull) + s);
+        mbar_arrive_expect_tx(fb, C::kHalfBytes);
+        for (int bx = 0; bx < C::kBoxes; ++bx)
+          tma_load_3d((half ? sDO(s) : sQ(s)) + bx * C::kBoxBytes, half ? &tm_do : &tm_q, fb, bx * 64,
+                      q0, bh_q);
         const size_t voff = (size_t)bh_q * p.nq_pad + q0;
-        bulk_load(base + C::kOffVec + s * kBQ * 4, p.lse2 + voff, kBQ * 4, fb);
-        bulk_load(base + C::kOffVec + (2 + s) * kBQ * 4, p.dvec + voff, kBQ * 4, fb);
+        bulk_load(base + C::kOffVec + (2 * half + s) * kBQ * 4, (half ? p.dvec : p.lse2) + voff,
+                  kBQ * 4, fb);
       }
       __syncwarp();
     }
     if (!ok) {
       if (lane == 0) {
         flag_abort(abort_flag, p.status, 0x100 | (it << 12));
-        // let the loads in flight land before the CTA exits
+        // let the loads in flight land before the CTA exits (loads issued:
+        // both halves of blocks < it, and the Q half of block it if half = 1)
         volatile int no_abort = 0;
         bounded_wait(bar(Bars::kKV), 0, &no_abort, budget);
-        for (int i = max(0, it - 2); i < it; ++i)
-          bounded_wait(bar(Bars::kFull + (i & 1)), (i >> 1) & 1, &no_abort, budget);
+        for (int i = max(0, it - 2); i <= it && i < n_iter; ++i) {
+          if (i < it || half) bounded_wait(bar(Bars::kFull + (i & 1)), (i >> 1) & 1, &no_abort, budget);
+          if (i < it) bounded_wait(bar(Bars::kFullDO + (i & 1)), (i >> 1) & 1, &no_abort, budget);
+        }
       }
       __syncwarp();
     }
@@ -311,7 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tDV = tmem + C::kColDV, tDK = tmem + C::kColDK;
     int it = 0;
     bool ok = warp_all(bounded_wait(bar(Bars::kKV), 0, abort_flag, budget) &&
-                       bounded_wait(bar(Bars::kFull + 0), 0, abort_flag, budget));
+                       bounded_wait(bar(Bars::kFull + 0), 0, abort_flag, budget) &&
+                       bounded_wait(bar(Bars::kFullDO + 0), 0, abort_flag, budget));
     if (ok) {
       tc_fence_after();
       if (lane == 0) {
@@ -351,7 +369,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (more) {
-        ok = warp_all(bounded_wait(bar(Bars::kDQFree), it & 1, abort_flag, budget));
+        ok = warp_all(bounded_wait(bar(Bars::kDQFree), it & 1, abort_flag, budget) &&
+                      bounded_wait(bar(Bars::kFullDO + (s ^ 1)), ((it + 1) >> 1) & 1, abort_flag, budget));
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
@@ -431,7 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(Bars::kP));
 
-      ok = warp_all(bounded_wait(bar(Bars::kDP), it & 1, abort_flag, budget));
+      ok = warp_all(bounded_wait(bar(Bars::kFullDO + s), (it >> 1) & 1, abort_flag, budget) &&
+                    bounded_wait(bar(Bars::kDP), it & 1, abort_flag, budget));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
@@ -479,7 +499,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int it = 0;
     for (; it < n_iter; ++it) {
-      ok = warp_all(bounded_wait(bar(Bars::kDQ), it & 1, abort_flag, budget));
+      // the four drain warps meet at named barriers below, which cannot time
+      // out: they decide together whether to go on
+      ok = named_bar_and(1, 128, bounded_wait(bar(Bars::kDQ), it & 1, abort_flag, budget));
       if (!ok) break;
       tc_fence_after();
       uint32_t v[D];
@@ -488,16 +510,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(Bars::kDQFree));
+      // Stage dQ(it) in the dO buffer of its stage (free: dP(it) and dV(it)
+      // completed before dQ(it)) 16 KB = 32 columns at a time, alternating
+      // kStageBufs buffers, each chunk added into the accumulator by one bulk
+      // reduce. Accumulator layout per 128-row block: [d/4][128 rows][4].
+      const int s = it & 1;
       const int q0 = q_block(it) * kBQ;
-      if (q0 + wq * 32 < p.Nq) {
-        // accumulator layout [B*Hq][Nq_pad/32][d/4][32][4]: a warp's 32 rows of
-        // one 4-column group are 512 contiguous bytes
-        const int bh_q = b * p.Hq + q_head(it);
-        float* acc = p.dq_acc + (((size_t)bh_q * (p.nq_pad / 32) + (q0 / 32 + wq)) * (D / 4)) * 128 + lane * 4;
+      const int bh_q = b * p.Hq + q_head(it);
+      float* const acc = p.dq_acc + ((size_t)bh_q * (p.nq_pad / kBQ) + q0 / kBQ) * kBQ * D;
+      uint8_t* const stage = base_ptr + C::kOffDO + s * 2 * C::kTileBytes;
+      const int r = wq * 32 + lane;
+      const bool leader = warp == 4 && lane == 0;
 #pragma unroll
-        for (int c4 = 0; c4 < D / 4; ++c4)
-          red_add_v4(acc + c4 * 128, __uint_as_float(v[4 * c4]), __uint_as_float(v[4 * c4 + 1]),
-                     __uint_as_float(v[4 * c4 + 2]), __uint_as_float(v[4 * c4 + 3]));
+      for (int q = 0; q < D / 32; ++q) {
+        uint8_t* const buf = stage + (q % C::kStageBufs) * 16384;
+        if (q >= C::kStageBufs) {
+          // the chunk that used this buffer must have been read
+          if (leader) bulk_wait_read<C::kStageBufs - 1>();
+          named_bar_sync(1, 128);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int g = 8 * q + c;
+          *reinterpret_cast<float4*>(buf + c * 2048 + r * 16) =
+              make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
+                          __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (leader) {
+          bulk_reduce_add_f32(acc + q * 4096, smem_addr(buf), 16384);
+          tma_store_commit();
+        }
+      }
+      if (leader) {
+        bulk_wait_read<0>();
+        mbar_arrive(bar(Bars::kEmptyDO + s));
       }
     }
     if (ok) ok = warp_all(bounded_wait(bar(Bars::kAcc), 0, abort_flag, budget));
@@ -559,23 +607,26 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const BwdPreParams p)
     }
     p.lse2[v] = l2;
   }
-  // the 32-row group of the accumulator is 32 * D contiguous floats
-  float4* acc_rows = reinterpret_cast<float4*>(p.dq_acc + ((size_t)bh * (p.nq_pad / 32) + g) * 32 * D);
+  // zero the accumulator's floats [32 D g, 32 D (g + 1)) of this head (the
+  // groups of a head together cover its nq_pad * D floats, whatever the layout)
+  float4* acc_rows = reinterpret_cast<float4*>(p.dq_acc + ((size_t)bh * p.nq_pad + g * 32) * D);
   for (int i = threadIdx.x; i < 8 * D; i += 256) acc_rows[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // dQ = bf16(scale * accumulator), through a shared-memory transpose so both
-// the accumulator reads and the dQ row writes are contiguous.
+// the accumulator reads and the dQ row writes are contiguous. The accumulator
+// holds each 128-row block as [d/4][128 rows][4]; a CTA converts 32 rows.
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_post_kernel(const BwdPostParams p) {
   constexpr int kPitch = D + 8;  // bf16 elements per staged row (breaks bank conflicts)
   __shared__ __align__(16) uint16_t tile[32 * kPitch];
   const int g = blockIdx.x;
   const int bh = blockIdx.y;
-  const float4* src = reinterpret_cast<const float4*>(p.dq_acc + ((size_t)bh * (p.nq_pad / 32) + g) * 32 * D);
+  const float4* src = reinterpret_cast<const float4*>(p.dq_acc + ((size_t)bh * p.nq_pad + (g >> 2) * kBQ) * D) +
+                      (g & 3) * 32;
   for (int i = threadIdx.x; i < 8 * D; i += 256) {
-    const float4 a = src[i];
     const int c4 = i >> 5, row = i & 31;
+    const float4 a = src[c4 * kBQ + row];
     uint2 w;
     w.x = pack_bf16x2(a.x * p.scale, a.y * p.scale);
     w.y = pack_bf16x2(a.z * p.scale, a.w * p.scale);

@@ -67,7 +67,7 @@ cudaError_t launch_q8(const Q8Launch& L, int d, cudaStream_t stream);
 struct BwdParams {
   void* dk;                       // bf16 [B, Hkv, Nkv, d]
   void* dv;                       // bf16 [B, Hkv, Nkv, d]
-  float* dq_acc;                  // fp32 [B*Hq][nq_pad/32][d/4][32][4]
+  float* dq_acc;                  // fp32 [B*Hq][nq_pad/128][d/4][128][4]
   const float* lse2;              // fp32 [B*Hq][nq_pad]  LSE * log2(e), +inf where P must be 0
   const float* dvec;              // fp32 [B*Hq][nq_pad]  D_i = sum_c dO_ic O_ic
   int* status;
