@@ -33,7 +33,7 @@ from synthetic import (VARLEN_WORKLOADS, WORKLOADS, Workload, bf16_bits, make_do
                        make_varlen)
 
 HEADLINE = "outlier_8k_causal"
-EXTRA_BF16 = ["causal_2k_d128", "outlier_8k_full", "gqa_32k_d128", "gqa_32k_d64"]
+EXTRA_BF16 = ["causal_2k_d128", "outlier_8k_full", "gqa_32k_d128", "gqa_32k_d64", "d256_8k_causal"]
 METRIC = "attn fwd TFLOP/s (4·B·H·N²·d, causal halved), % of B200 dense BF16 peak"
 L2_BYTES = 126 * 2 ** 20
 KERNEL_SOURCES = ["exact_attention_134_b200/csrc/attn_fwd_sm100.cu",

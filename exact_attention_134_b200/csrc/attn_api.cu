@@ -71,16 +71,18 @@ int device_sm_count() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// d = 96 is supported by the bf16 kernels only (allow96 = false for the 8-bit paths).
+// d = 96 is supported by the bf16 kernels only (allow96 = false for the 8-bit
+// paths and the backward); d = 256 by the dense bf16 forward only (allow256).
 attn_status_t check_args(const void* q, const void* k, const void* v, const void* o,
                          const void* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
-                         int causal, float scale, bool allow96 = true) {
+                         int causal, float scale, bool allow96 = true, bool allow256 = false) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nkv <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.0f)) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128 && !(allow96 && d == 96)) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && !(allow96 && d == 96) && !(allow256 && d == 256))
+    return ATTN_ERR_UNSUPPORTED;
   if (B > 65535 || Hq > 65535) return ATTN_ERR_UNSUPPORTED;
   // TMA global strides must stay below 2^40 bytes.
   const unsigned long long head_bytes_q = 2ull * (unsigned long long)Nq * d;
@@ -94,10 +96,11 @@ attn_status_t check_args(const void* q, const void* k, const void* v, const void
 // bf16 tensor [BH, N, d] as a 3-D map {d, N, BH}; box = 64 columns x 128 rows,
 // 128-byte swizzle (the layout the tcgen05 descriptors expect).
 // (d = 96: 32-column boxes with the 64-byte swizzle, three per 96-column row.)
+// (d = 256 K/V: 64-row boxes, the d = 256 kernel's 64-key tiles.)
 bool make_map(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * (cuuint64_t)d * 2};
-  cuuint32_t box[3] = {d == 96 ? 32u : 64u, 128, 1};
+  cuuint32_t box[3] = {d == 96 ? 32u : 64u, d == 256 ? 64u : 128u, 1};
   cuuint32_t elem_strides[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
                         strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -139,9 +142,14 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   int* status = device_status_ptr();
   if (!status) return ATTN_ERR_CUDA;
   alignas(64) CUtensorMap tq, tk, tv, to;
-  if (!make_map(&tq, q, d, Nq, (long long)B * Hq) || !make_map(&tk, k, d, Nkv, (long long)B * Hkv) ||
-      !make_map(&tv, v, d, Nkv, (long long)B * Hkv) || !make_map(&to, o, d, Nq, (long long)B * Hq))
+  if (d == 256) {
+    if (!make_map(&tk, k, d, Nkv, (long long)B * Hkv) || !make_map(&tv, v, d, Nkv, (long long)B * Hkv))
+      return ATTN_ERR_CUDA;
+  } else if (!make_map(&tq, q, d, Nq, (long long)B * Hq) ||
+             !make_map(&tk, k, d, Nkv, (long long)B * Hkv) ||
+             !make_map(&tv, v, d, Nkv, (long long)B * Hkv) || !make_map(&to, o, d, Nq, (long long)B * Hq)) {
     return ATTN_ERR_CUDA;
+  }
   attn_sm100::FwdParams p;
   p.o = o;
   p.lse = lse;
@@ -166,6 +174,7 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
 #endif
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
+  if (d == 256) return cuda_status(attn_sm100::launch_fwd_d256(tk, tv, q, p, stream));
   return cuda_status(attn_sm100::launch_fwd_bf16(tq, tk, tv, to, p, d, stream));
 }
 
@@ -392,7 +401,7 @@ extern "C" {
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                        int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
                        void* stream) {
-  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, true, true);
   if (s != ATTN_OK) return s;
   return run_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale,
                  static_cast<cudaStream_t>(stream));
@@ -423,8 +432,8 @@ attn_status_t attn_fwd_host(const void* q_host, const void* k_host, const void* 
                             void* o_host, float* lse_host, int B, int Hq, int Hkv, int Nq, int Nkv,
                             int d, int causal, float scale, void* dev_buf, size_t dev_buf_bytes,
                             void* stream) {
-  attn_status_t s =
-      check_args(q_host, k_host, v_host, o_host, lse_host, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  attn_status_t s = check_args(q_host, k_host, v_host, o_host, lse_host, B, Hq, Hkv, Nq, Nkv, d,
+                               causal, scale, true, true);
   if (s != ATTN_OK) return s;
   if (!dev_buf || !aligned16(dev_buf)) return ATTN_ERR_WORKSPACE;
   const HostLayout L = host_layout(B, Hq, Hkv, Nq, Nkv, d);

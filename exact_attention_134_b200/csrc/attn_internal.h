@@ -119,4 +119,9 @@ cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t stream);
 int fwd_rows_per_cta();
 
+// Head dim 256 (dense tensors only): K/V tensor maps with 64-row boxes; Q is
+// read directly from global memory.
+cudaError_t launch_fwd_d256(const CUtensorMap& tk, const CUtensorMap& tv, const void* q,
+                            const FwdParams& p, cudaStream_t stream);
+
 }  // namespace attn_sm100

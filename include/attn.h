@@ -21,7 +21,10 @@
  *     mask is aligned to the bottom right (for Nq == Nkv: j <= i; for Nq < Nkv
  *     a prefill whose first Nkv - Nq keys are a cache). A row that sees no
  *     key (only possible when Nq > Nkv) gets O = 0 and LSE = -inf.
- *   - Head dim d is 64, 96 or 128 (the 8-bit entry points: 64 or 128).
+ *   - Head dim d is 64, 96 or 128; attn_fwd and attn_fwd_host also take 256
+ *     (the "FlashAttention-2 (2023)" section's largest head dimension; its own
+ *     kernel: one query tile per CTA, Q held in tensor memory); the 8-bit
+ *     entry points and the backward take 64 or 128.
  *   - Ownership: the caller owns every buffer; device pointers must stay valid
  *     until the work queued on `stream` has finished. The library allocates no
  *     device memory. `stream` is a cudaStream_t (0 = legacy default stream).
@@ -54,7 +57,7 @@ extern "C" {
 typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_INVALID_ARG = 1,  /* NULL pointer, a size <= 0, Hq % Hkv != 0, scale not finite or <= 0 */
-  ATTN_ERR_UNSUPPORTED = 2,  /* d not in {64, 96, 128} (8-bit: {64, 128}); B, Hq or sequence count > 65535; a head beyond 2^40 bytes */
+  ATTN_ERR_UNSUPPORTED = 2,  /* d not supported by the entry point (see "Head dim"); B, Hq or sequence count > 65535; a head beyond 2^40 bytes */
   ATTN_ERR_ALIGNMENT = 3,    /* a device pointer is not 16-byte aligned */
   ATTN_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (no device, launch failure, ...) */
   ATTN_ERR_TIMEOUT = 5,      /* a kernel pipeline wait exceeded its budget (reported by attn_get_status) */

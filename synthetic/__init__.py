@@ -77,6 +77,9 @@ WORKLOADS = {
                               dist="outlier_k", path="q8", oracle_rows=64),
     "q8_8k_normal": Workload("q8_8k_normal", 2, 32, 32, 8192, 8192, 128, True, 1006,
                              path="q8", oracle_rows=64),
+    # head dim 256 (the largest the FlashAttention-2 section names), 8k causal
+    "d256_8k_causal": Workload("d256_8k_causal", 1, 16, 16, 8192, 8192, 256, True, 1008,
+                               oracle_rows=64),
 }
 
 

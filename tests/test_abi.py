@@ -53,7 +53,7 @@ def _fwd(lib, q=P, k=P, v=P, o=P, lse=P, B=1, Hq=2, Hkv=2, Nq=128, Nkv=128, d=12
     (dict(q=0), 1), (dict(lse=0), 1), (dict(B=0), 1), (dict(Nq=0), 1), (dict(Nkv=-1), 1),
     (dict(Hq=3, Hkv=2), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1),
     (dict(scale=float("inf")), 1), (dict(scale=-1.0), 1), (dict(causal=2), 1),
-    (dict(d=80), 2), (dict(d=256), 2), (dict(B=70000), 2),
+    (dict(d=80), 2), (dict(d=512), 2), (dict(d=32), 2), (dict(B=70000), 2),
     (dict(q=P + 2), 3), (dict(o=P + 8), 3), (dict(lse=P + 4), 3),
 ])
 def test_argument_validation(lib, kw, code):
@@ -96,6 +96,7 @@ def test_q8_entry_validation(lib):
     assert lib.attn_fwd_q8(*args, P, need - 1, None) == 6
     assert lib.attn_fwd_q8(P, P, P, P, P, 1, 2, 2, 300, 300, 96, 0, 0.125, P, need, None) == 2
     assert lib.attn_fwd_fp8(P, P, P, P, P, 1, 2, 2, 300, 300, 96, 0, 0.125, P, need, None) == 2
+    assert lib.attn_fwd_q8(P, P, P, P, P, 1, 2, 2, 300, 300, 256, 0, 0.125, P, need, None) == 2
     assert lib.attn_q8_prepass(P, P, P, 1, 2, 2, 300, 300, 128, None, need, None) == 6
     assert lib.attn_q8_workspace_offsets(0, 2, 2, 300, 300, 128, off) == 1
 
@@ -106,7 +107,7 @@ def test_varlen_entry_validation(lib):
     assert call(cq=None) == 1 and call(ck=None) == 1
     assert call(n=0) == 1 and call(mq=0) == 1 and call(tq=0) == 1 and call(Hq=3) == 1
     assert call(scale=float("nan")) == 1 and call(causal=3) == 1
-    assert call(d=80) == 2 and call(n=70000) == 2
+    assert call(d=80) == 2 and call(d=256) == 2 and call(n=70000) == 2
     assert call(q=P + 2) == 3 and call(cq=P + 2) == 3
 
 
@@ -122,6 +123,6 @@ def test_bwd_entry_validation(lib):
                             ws, nbytes, None)
     assert call(dq=None) == 1 and call(dout=None) == 1 and call(Hq=3) == 1
     assert call(causal=2) == 1 and call(scale=-1.0) == 1
-    assert call(d=96) == 2 and call(B=40000, Hq=4) == 2
+    assert call(d=96) == 2 and call(d=256) == 2 and call(B=40000, Hq=4) == 2
     assert call(dq=P + 4) == 3
     assert call(ws=None) == 6 and call(ws=P + 8) == 6 and call(nbytes=need - 1) == 6

@@ -85,6 +85,13 @@ SMALL = [
     (2, 8, 1, 513, 513, 96, True),
     (1, 2, 2, 100, 777, 96, False),
     (1, 2, 2, 200, 650, 96, True),
+    # head dim 256: one query tile per CTA, Q held in TMEM, 64-key K/V tiles
+    (1, 2, 2, 256, 256, 256, False),
+    (1, 1, 1, 1, 1, 256, True),
+    (1, 4, 2, 300, 300, 256, True),
+    (2, 2, 1, 129, 700, 256, False),
+    (1, 4, 4, 1000, 1000, 256, True),
+    (1, 2, 2, 64, 65, 256, True),
 ]
 
 
@@ -103,7 +110,8 @@ def test_causal_2k_workload():
     _check(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.causal, w.seed)
 
 
-@pytest.mark.parametrize("name", ["outlier_8k_causal", "outlier_8k_full", "gqa_32k_d128", "gqa_32k_d64"])
+@pytest.mark.parametrize("name", ["outlier_8k_causal", "outlier_8k_full", "gqa_32k_d128", "gqa_32k_d64",
+                                  "d256_8k_causal"])
 def test_large_workloads_sampled_rows(name):
     w = WORKLOADS[name]
     _check(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.causal, w.seed, w.dist, n_rows=w.oracle_rows)

@@ -45,6 +45,7 @@ def _check(og, lg, O, L, packed=False):
 @pytest.mark.parametrize("shape", [
     (1, 4, 2, 100, 333, 128), (1, 2, 2, 300, 1000, 64), (2, 4, 4, 513, 1537, 128),
     (1, 2, 2, 1, 700, 128), (1, 2, 2, 300, 100, 128), (1, 4, 1, 257, 129, 64),
+    (1, 2, 2, 500, 130, 256), (1, 4, 2, 100, 333, 256),
 ])
 def test_causal_bottom_right_dense(shape):
     B, Hq, Hkv, Nq, Nkv, d = shape
