@@ -9,6 +9,7 @@ missing or cannot run, the call raises.
 
     o, lse = attn_fwd(q, k, v, causal=True)          # bf16 [B,H,N,d] on cuda
     dq, dk, dv = attn_bwd(q, k, v, o, lse, do, causal=True)
+    o = attention(q, k, v, causal=True); o.backward(do)  # torch autograd
 """
 from __future__ import annotations
 
@@ -203,6 +204,41 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
                         _stream_handle(q.device))
     _check(st, "attn_bwd")
     return dq, dk, dv
+
+
+_AUTOGRAD_FN = None
+
+
+def _autograd_fn():
+    """torch.autograd.Function over attn_fwd / attn_bwd (created on first use
+    so that importing this module does not import torch)."""
+    global _AUTOGRAD_FN
+    if _AUTOGRAD_FN is None:
+        import torch
+
+        class _Attention(torch.autograd.Function):
+            @staticmethod
+            def forward(ctx, q, k, v, causal, scale):
+                o, lse = attn_fwd(q, k, v, causal=causal, scale=scale)
+                ctx.save_for_backward(q, k, v, o, lse)
+                ctx.causal, ctx.scale = causal, scale
+                return o
+
+            @staticmethod
+            def backward(ctx, do):
+                q, k, v, o, lse = ctx.saved_tensors
+                dq, dk, dv = attn_bwd(q, k, v, o, lse, do.contiguous(), causal=ctx.causal, scale=ctx.scale)
+                return dq, dk, dv, None, None
+
+        _AUTOGRAD_FN = _Attention
+    return _AUTOGRAD_FN
+
+
+def attention(q, k, v, causal: bool = False, scale: float | None = None):
+    """Differentiable exact attention for training: the forward is attn_fwd
+    (O only; LSE is kept for the backward), the backward attn_bwd. Same
+    tensors and head dims as attn_bwd (d = 64 or 128)."""
+    return _autograd_fn().apply(q, k, v, causal, scale)
 
 
 def q8_workspace_size(B, Hq, Hkv, Nq, Nkv, d) -> int:

@@ -225,3 +225,22 @@ def test_bwd_full_size_sampled():
                            q_rows=np.stack([rows[b, h] for b, h in heads])[:, None], kv_rows=kv_rows,
                            dq=sl(dq.cpu()), dk=sl(dk.cpu()), dv=sl(dv.cpu()), vacuous=0.3)
     assert worst <= 1.0
+
+
+def test_autograd_function_matches_torch_fp32():
+    """attention() as a torch.autograd.Function: gradients of a scalar loss
+    through it against torch's own autograd of the fp32 definition."""
+    B, Hq, Hkv, N, d = 1, 4, 2, 300, 128
+    q, k, v = make_qkv(B, Hq, Hkv, N, N, d, seed=31)
+    qc, kc, vc = (t.cuda().requires_grad_() for t in (q, k, v))
+    o = attn.attention(qc, kc, vc, causal=True)
+    w = make_dout(B, Hq, N, d, seed=31).cuda()
+    (o.float() * w.float()).sum().backward()
+    qf, kf, vf = (t.cuda().float().requires_grad_() for t in (q, k, v))
+    mask = torch.ones(N, N, dtype=torch.bool, device="cuda").tril()
+    of = torch.nn.functional.scaled_dot_product_attention(
+        qf, kf.repeat_interleave(2, 1), vf.repeat_interleave(2, 1), attn_mask=mask)
+    (of * w.float()).sum().backward()
+    for a, r in ((qc.grad, qf.grad), (kc.grad, kf.grad), (vc.grad, vf.grad)):
+        assert a.dtype == torch.bfloat16 and a.shape == r.shape
+        assert (a.float() - r).abs().max().item() <= 2e-2 * r.abs().max().item()
