@@ -2,6 +2,7 @@
 // tensor-map (TMA descriptor) construction, launch, device status word.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -290,6 +291,40 @@ struct HostLayout {
   size_t q, k, v, o, lse, total;
 };
 
+// Streams and events of the host-buffer entry point, created once per device
+// (with that device current) and kept for the process: a copy-in stream, a
+// copy-out stream and the per-chunk events that order them around the caller's
+// stream, on which the kernels run.
+constexpr int kHostChunks = 8;
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t loaded[kHostChunks] = {}, computed[kHostChunks] = {};
+  bool ready = false;
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_pipe_mutex[kMaxDevices];  // one enqueue sequence at a time per device
+
+HostPipe* host_pipe() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  HostPipe& P = g_pipe[dev];
+  if (!P.ready) {
+    const unsigned f = cudaEventDisableTiming;
+    bool ok = cudaStreamCreateWithFlags(&P.in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&P.out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&P.start, f) == cudaSuccess &&
+              cudaEventCreateWithFlags(&P.done, f) == cudaSuccess;
+    for (int i = 0; ok && i < kHostChunks; ++i)
+      ok = cudaEventCreateWithFlags(&P.loaded[i], f) == cudaSuccess &&
+           cudaEventCreateWithFlags(&P.computed[i], f) == cudaSuccess;
+    if (!ok) return nullptr;
+    P.ready = true;
+  }
+  return &P;
+}
+
 HostLayout host_layout(int B, int Hq, int Hkv, int Nq, int Nkv, int d) {
   HostLayout L;
   const size_t qo = 2ull * B * Hq * (size_t)Nq * d;
@@ -440,20 +475,60 @@ attn_status_t attn_fwd_host(const void* q_host, const void* k_host, const void* 
   if (dev_buf_bytes < L.total) return ATTN_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* base = static_cast<char*>(dev_buf);
-  const size_t qo = 2ull * B * Hq * (size_t)Nq * d;
-  const size_t kv = 2ull * B * Hkv * (size_t)Nkv * d;
-  if (cudaMemcpyAsync(base + L.q, q_host, qo, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(base + L.k, k_host, kv, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(base + L.v, v_host, kv, cudaMemcpyHostToDevice, st) != cudaSuccess)
-    return ATTN_ERR_CUDA;
-  s = run_fwd(base + L.q, base + L.k, base + L.v, base + L.o, reinterpret_cast<float*>(base + L.lse),
-              B, Hq, Hkv, Nq, Nkv, d, causal, scale, st);
-  if (s != ATTN_OK) return s;
-  if (cudaMemcpyAsync(o_host, base + L.o, qo, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-      cudaMemcpyAsync(lse_host, base + L.lse, 4ull * B * Hq * (size_t)Nq, cudaMemcpyDeviceToHost,
-                      st) != cudaSuccess)
-    return ATTN_ERR_CUDA;
-  return cudaStreamSynchronize(st) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  HostPipe* P = host_pipe();
+  if (!P || !device_status_ptr()) return ATTN_ERR_CUDA;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  // Pipeline over chunks of whole kv-head groups (flattened over batch and
+  // heads, so each chunk is contiguous in every tensor): chunk c's inputs are
+  // copied on P->in while chunk c-1 computes on `st` and chunk c-2's outputs
+  // are copied back on P->out. Each chunk is attn_fwd on a sub-problem with
+  // B = 1, Hq = its query heads, Hkv = its kv heads.
+  const int G = Hq / Hkv;
+  const long long groups = (long long)B * Hkv;
+  const int n_chunks = (int)std::min<long long>(kHostChunks, groups);
+  if ((groups + n_chunks - 1) / n_chunks * G > 65535) return ATTN_ERR_UNSUPPORTED;  // grid y of a chunk
+  const size_t q_head = 2ull * Nq * d, kv_head = 2ull * Nkv * d, lse_head = 4ull * Nq;
+  const char* qh = static_cast<const char*>(q_host);
+  const char* kh = static_cast<const char*>(k_host);
+  const char* vh = static_cast<const char*>(v_host);
+  char* oh = static_cast<char*>(o_host);
+  char* lh = reinterpret_cast<char*>(lse_host);
+  auto fail = [&](cudaError_t e) { return e == cudaSuccess ? ATTN_OK : cuda_status(e); };
+  std::unique_lock<std::mutex> lock(g_pipe_mutex[dev]);
+  cudaError_t e = cudaEventRecord(P->start, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(P->in, P->start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(P->out, P->start, 0);
+  if (e != cudaSuccess) return fail(e);
+  for (int c = 0; c < n_chunks; ++c) {
+    const long long g0 = groups * c / n_chunks, g1 = groups * (c + 1) / n_chunks;
+    const long long h0 = g0 * G, nh = (g1 - g0) * G, nk = g1 - g0;
+    e = cudaMemcpyAsync(base + L.q + h0 * q_head, qh + h0 * q_head, nh * q_head, cudaMemcpyHostToDevice, P->in);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(base + L.k + g0 * kv_head, kh + g0 * kv_head, nk * kv_head, cudaMemcpyHostToDevice, P->in);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(base + L.v + g0 * kv_head, vh + g0 * kv_head, nk * kv_head, cudaMemcpyHostToDevice, P->in);
+    if (e == cudaSuccess) e = cudaEventRecord(P->loaded[c], P->in);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, P->loaded[c], 0);
+    if (e != cudaSuccess) return fail(e);
+    s = run_fwd(base + L.q + h0 * q_head, base + L.k + g0 * kv_head, base + L.v + g0 * kv_head,
+                base + L.o + h0 * q_head, reinterpret_cast<float*>(base + L.lse + h0 * lse_head), 1,
+                (int)nh, (int)nk, Nq, Nkv, d, causal, scale, st);
+    if (s != ATTN_OK) return s;
+    e = cudaEventRecord(P->computed[c], st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(P->out, P->computed[c], 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(oh + h0 * q_head, base + L.o + h0 * q_head, nh * q_head, cudaMemcpyDeviceToHost, P->out);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(lh + h0 * lse_head, base + L.lse + h0 * lse_head, nh * lse_head,
+                          cudaMemcpyDeviceToHost, P->out);
+    if (e != cudaSuccess) return fail(e);
+  }
+  e = cudaEventRecord(P->done, P->out);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, P->done, 0);
+  lock.unlock();
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  return fail(e);
 }
 
 size_t attn_fwd_q8_workspace_size(int B, int Hq, int Hkv, int Nq, int Nkv, int d) {

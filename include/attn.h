@@ -104,9 +104,14 @@ ATTN_API attn_status_t attn_fwd_varlen(const void* q, const void* k, const void*
  * attn_fwd_host — the same operation on HOST buffers, for callers whose data
  * lives in host memory. Copies q, k, v into `dev_buf` (a device buffer of at
  * least attn_fwd_host_buffer_size() bytes, 16-byte aligned, owned by the
- * caller), runs attn_fwd on `stream`, copies o and lse back and synchronises
- * `stream` before returning. Host buffers should be page-locked for the copies
- * to run at full speed (pageable memory works, slower).
+ * caller), runs attn_fwd, copies o and lse back and synchronises `stream`
+ * before returning. The work is pipelined over up to 8 chunks of whole
+ * kv-head groups: chunk c's inputs are copied in while chunk c-1 is computed
+ * on `stream` and chunk c-2's outputs are copied out, on two copy streams the
+ * library creates once per device (with events that order them after the work
+ * already queued on `stream`). Host buffers should be page-locked for the
+ * copies to overlap and run at full speed (pageable memory works, slower).
+ * ATTN_ERR_UNSUPPORTED if a chunk would hold more than 65535 query heads.
  */
 ATTN_API size_t attn_fwd_host_buffer_size(int B, int Hq, int Hkv, int Nq, int Nkv, int d);
 ATTN_API attn_status_t attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,

@@ -176,3 +176,16 @@ def test_host_buffer_entry_point():
     O, L = oracle.attention_fp64(bf16_bits(q), bf16_bits(k), bf16_bits(v), True, 1 / 8)
     mx, mean, dl = _compare(o, lse, O, L)
     assert mx <= MAX_TOL and mean <= MEAN_TOL and dl <= LSE_TOL
+
+
+def test_host_entry_pipelined_chunks_match_device_entry():
+    """attn_fwd_host splits the work into chunks of kv-head groups (8 here,
+    GQA 4:1, two batch entries) and must give exactly attn_fwd's result."""
+    q, k, v = make_qkv(2, 16, 4, 700, 700, 128, seed=12)
+    o_h, l_h = attn.attn_fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), causal=True)
+    o_d, l_d = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True)
+    assert torch.equal(o_h, o_d.cpu()) and torch.equal(l_h, l_d.cpu())
+    q1, k1, v1 = make_qkv(1, 3, 1, 129, 300, 256, seed=13)  # one group: one chunk, d = 256
+    o_h, l_h = attn.attn_fwd_host(q1.pin_memory(), k1.pin_memory(), v1.pin_memory(), causal=False)
+    o_d, l_d = attn.attn_fwd(q1.cuda(), k1.cuda(), v1.cuda(), causal=False)
+    assert torch.equal(o_h, o_d.cpu()) and torch.equal(l_h, l_d.cpu())
