@@ -33,7 +33,8 @@ from synthetic import (VARLEN_WORKLOADS, WORKLOADS, Workload, bf16_bits, make_do
                        make_varlen)
 
 HEADLINE = "outlier_8k_causal"
-EXTRA_BF16 = ["causal_2k_d128", "outlier_8k_full", "gqa_32k_d128", "gqa_32k_d64", "d256_8k_causal"]
+EXTRA_BF16 = ["tiny_256_d64", "causal_2k_d128", "outlier_8k_full", "gqa_32k_d128", "gqa_32k_d64",
+              "d256_8k_causal"]
 METRIC = "attn fwd TFLOP/s (4·B·H·N²·d, causal halved), % of B200 dense BF16 peak"
 L2_BYTES = 126 * 2 ** 20
 KERNEL_SOURCES = ["exact_attention_134_b200/csrc/attn_fwd_sm100.cu",
@@ -413,8 +414,12 @@ def run_ours(args):
             r = bench_workload(wx, max(3, args.steps // 2), 3, world, rank, attn)
             msx = r["total_ms"] / max(3, args.steps // 2)
             tf = world * wx.flops / (msx * 1e-3) / 1e12
+            gbs = world * wx.min_hbm_bytes / (msx * 1e-3) / 1e9
             extras[name] = {"tflops": round(tf, 1), "ms_per_step": round(msx, 4),
+                            "us_per_step": round(msx * 1e3, 2),
                             "frac_of_bf16_peak": round(tf / world / peaks["bf16"], 4),
+                            "hbm_gbs_algorithmic": round(gbs, 1),
+                            "frac_of_hbm_peak": round(gbs / world / peaks["hbm"], 4),
                             "l2": r["l2"]}
             del r
             torch.cuda.empty_cache()
@@ -451,6 +456,8 @@ def run_ours(args):
             "steps": args.steps,
             "warmup": max(args.warmup, 3),
             "ms_per_step": round(ms, 4),
+            "ms_min": round(min(res["times"]), 4),
+            "ms_median": round(statistics.median(res["times"]), 4),
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
