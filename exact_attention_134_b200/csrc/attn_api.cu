@@ -22,7 +22,6 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 std::mutex g_dev_mutex;
 int* g_status_ptr[kMaxDevices] = {nullptr};
-int g_sm_count[kMaxDevices] = {0};
 std::atomic<long long> g_timeout_ns{1000000000LL};
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
@@ -54,20 +53,9 @@ int* device_status_ptr() {
   if (!g_status_ptr[dev]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) return nullptr;
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-      return nullptr;
-    g_sm_count[dev] = sms;
     g_status_ptr[dev] = static_cast<int*>(ptr);
   }
   return g_status_ptr[dev];
-}
-
-// SM count of the current device (valid after device_status_ptr() succeeded).
-int device_sm_count() {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  return g_sm_count[dev];
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -165,14 +153,6 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.causal = causal;
   const int rows = attn_sm100::fwd_rows_per_cta();
   p.num_row_blocks = (Nq + rows - 1) / rows;
-  const long long units = (long long)B * Hq * p.num_row_blocks;
-  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  p.num_units = (int)units;
-#ifdef ATTN_ONE_UNIT_PER_CTA
-  p.num_ctas = p.num_units;
-#else
-  p.num_ctas = device_sm_count();
-#endif
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
   if (d == 256) return cuda_status(attn_sm100::launch_fwd_d256(tk, tv, q, p, stream));
@@ -203,8 +183,6 @@ attn_status_t run_fwd_varlen(const void* q, const void* k, const void* v, void* 
   p.causal = causal;
   const int rows = attn_sm100::fwd_rows_per_cta();
   p.num_row_blocks = (max_seqlen_q + rows - 1) / rows;
-  p.num_units = 0;
-  p.num_ctas = 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
   // the output map is unused by the packed path (rows are stored one by one)

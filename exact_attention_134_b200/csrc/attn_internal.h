@@ -20,8 +20,6 @@ struct FwdParams {
   int B, Nq, Nkv, Hq, Hkv;        // packed: B = sequences, Nq / Nkv = total rows
   int causal;
   int num_row_blocks;             // ceil(Nq / rows per work unit); packed: of the longest sequence
-  int num_units;                  // B * Hq * num_row_blocks
-  int num_ctas;                   // persistent grid size (SM count)
   float scale_log2;               // scale * log2(e)
   unsigned long long timeout_ns;  // budget of every pipeline wait
 };
