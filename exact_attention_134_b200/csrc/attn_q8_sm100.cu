@@ -240,20 +240,28 @@ __global__ void __launch_bounds__(kPrepThreads)
       svc[i] = sv[bh * D + vc * 8 + i];
       rsv[i] = __frcp_rn(svc[i]);
     }
+    // K and V rows are loaded raw (bf16) before the block-wide maximum, so that
+    // all of this thread's loads are in flight at once; they are unpacked
+    // where they are used
+    uint4 kraw[NP], vraw[NP];
+#pragma unroll
+    for (int pp = 0; pp < NP; ++pp) {
+      const int t = kb_i * kTok + rs + pp * RPP;
+      kraw[pp] = t < Nkv ? *reinterpret_cast<const uint4*>(k + (bh * Nkv + t) * D + vc * 8)
+                         : make_uint4(0, 0, 0, 0);
+      vraw[pp] = t < Nkv ? *reinterpret_cast<const uint4*>(v + (bh * Nkv + t) * D + vc * 8)
+                         : make_uint4(0, 0, 0, 0);
+    }
     float amax = 0.0f;
 #pragma unroll
     for (int pp = 0; pp < NP; ++pp) {
       const int t = kb_i * kTok + rs + pp * RPP;
       if (t < Nkv) {
-        unpack8(*reinterpret_cast<const uint4*>(k + (bh * Nkv + t) * D + vc * 8), x[pp]);
+        float xk[8];
+        unpack8(kraw[pp], xk);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) x[pp][i] = x[pp][i] - kb[i];
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[pp][i] = 0.0f;
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(xk[i] - kb[i]));
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[pp][i]));
     }
     amax = block_max256(amax, red);
     const float s = amax > 0.0f ? __fdiv_rn(amax, F8 ? 448.0f : 127.0f) : 1.0f;
@@ -262,9 +270,13 @@ __global__ void __launch_bounds__(kPrepThreads)
     for (int pp = 0; pp < NP; ++pp) {
       const int t = kb_i * kTok + rs + pp * RPP;
       if (t < Nkv) {
-        *reinterpret_cast<uint2*>(k8 + (bh * Nkv + t) * D + vc * 8) = codes8<F8>(x[pp], s, r_s);
+        float xk[8];
+        unpack8(kraw[pp], xk);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xk[i] = xk[i] - kb[i];
+        *reinterpret_cast<uint2*>(k8 + (bh * Nkv + t) * D + vc * 8) = codes8<F8>(xk, s, r_s);
         float vf[8];
-        unpack8(*reinterpret_cast<const uint4*>(v + (bh * Nkv + t) * D + vc * 8), vf);
+        unpack8(vraw[pp], vf);
         float y[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) y[i] = div_rn(vf[i], svc[i], rsv[i]);
