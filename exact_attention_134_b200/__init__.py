@@ -55,6 +55,7 @@ _SIGNATURES = {
     "attn_q8_workspace_offsets": (_c_int, [_c_int] * 6 + [ctypes.POINTER(_sz)]),
     "attn_bwd_workspace_size": (_sz, [_c_int] * 6),
     "attn_bwd": (_c_int, [_vp] * 9 + [_c_int] * 7 + [_c_float, _vp, _sz, _vp]),
+    "attn_selftest_wait_timeout": (_c_int, [_c_int, _vp]),
     "attn_get_status": (_c_int, [_vp]),
     "attn_get_status_ex": (_c_int, [_vp, ctypes.POINTER(_c_int)]),
     "attn_set_timeout_ms": (_c_int, [_c_int]),
@@ -323,6 +324,12 @@ def attn_fwd_host(q, k, v, causal: bool = False, scale: float | None = None, dev
                              dev_buf.data_ptr(), dev_buf.numel(), _stream_handle(dev_buf.device))
     _check(st, "attn_fwd_host")
     return out, lse
+
+
+def selftest_wait_timeout(budget_us: int) -> None:
+    """Queue the failure-detection self-test (a bounded wait that must time out
+    after budget_us and record ATTN_ERR_TIMEOUT, where = 0xF00)."""
+    _check(lib().attn_selftest_wait_timeout(int(budget_us), _stream_handle()), "attn_selftest_wait_timeout")
 
 
 def get_status(stream: int | None = None) -> tuple[int, int]:

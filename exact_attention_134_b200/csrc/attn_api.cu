@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "attn_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace {
 
@@ -190,6 +191,25 @@ attn_status_t run_fwd_varlen(const void* q, const void* k, const void* v, void* 
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Failure-detection self-test: one thread waits, with the kernels' own bounded
+// wait, on an mbarrier that nothing completes. The wait must give up after its
+// budget and record ATTN_ERR_TIMEOUT (where = 0xF00) in the status word; the
+// kernel then returns normally, so the context stays usable.
+__global__ void selftest_wait_timeout_kernel(int* status, unsigned long long budget_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    attn_sm100::mbar_init(attn_sm100::smem_addr(&bar), 1);
+    abort_flag = 0;
+    attn_sm100::fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 &&
+      !attn_sm100::bounded_wait(attn_sm100::smem_addr(&bar), 0, &abort_flag, budget_ns)) {
+    if (atomicCAS(status, 0, ATTN_ERR_TIMEOUT) == 0) status[1] = 0xF00;
+  }
+}
 
 // Workspace of the 8-bit path, in this order, each region 256-byte aligned:
 // q8, k8, v8 (1 byte per element), sq, sk, sv, kbar, qk (fp32), ksum partials
@@ -582,6 +602,15 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
     return ATTN_ERR_WORKSPACE;
   return run_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nkv, d, causal, scale,
                  workspace, static_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_selftest_wait_timeout(int budget_us, void* stream) {
+  if (budget_us < 1 || budget_us > 10000000) return ATTN_ERR_INVALID_ARG;
+  int* status = device_status_ptr();
+  if (!status) return ATTN_ERR_CUDA;
+  selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      status, 1000ull * (unsigned long long)budget_us);
+  return cuda_status(cudaGetLastError());
 }
 
 attn_status_t attn_get_status_ex(void* stream, int* where) {

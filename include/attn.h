@@ -256,6 +256,18 @@ ATTN_API attn_status_t attn_get_status(void* stream);
  * (0 when nothing failed). */
 ATTN_API attn_status_t attn_get_status_ex(void* stream, int* where);
 
+/*
+ * attn_selftest_wait_timeout — exercises the failure-detection path without a
+ * fault: one GPU thread waits, with the same bounded wait the kernels use, on
+ * a barrier that nothing completes; after `budget_us` microseconds (1 ..
+ * 10^7) it gives up and records ATTN_ERR_TIMEOUT in the device status word
+ * (where = 0xF00), and the kernel returns normally. Read the result with
+ * attn_get_status_ex(). Queued on `stream`; ATTN_ERR_INVALID_ARG for a budget
+ * outside the range. Not part of the method: a test hook for the timeout
+ * machinery every attention kernel relies on.
+ */
+ATTN_API attn_status_t attn_selftest_wait_timeout(int budget_us, void* stream);
+
 /* attn_set_timeout_ms — budget of every in-kernel pipeline wait (default 1000
  * ms; values < 1 are rejected with ATTN_ERR_INVALID_ARG). Process-wide. */
 ATTN_API attn_status_t attn_set_timeout_ms(int ms);
