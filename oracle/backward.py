@@ -95,3 +95,28 @@ def attention_bwd_head(q, k, v, do, causal: bool, scale: float, block_rows: int 
         dK += scale * (blk["dS"].T @ q[i0:i1])
         dV += blk["P"].T @ do[i0:i1]
     return dQ, dK, dV
+
+
+def attention_varlen_bwd_fp64(q_bits, k_bits, v_bits, do_bits, cu_q, cu_k, causal: bool,
+                              scale: float):
+    """Backward of attention_varlen_fp64: packed sequences q, do [total_q, Hq, d],
+    k, v [total_k, Hkv, d] (uint16 bf16 bits), sequence s owning query rows
+    cu_q[s]:cu_q[s+1] and key rows cu_k[s]:cu_k[s+1]; each sequence is the
+    dense backward on its own rows (causal mask bottom-right per sequence).
+    Returns float64 (dQ, dK, dV) in the packed layouts."""
+    total_q, Hq, d = q_bits.shape
+    total_k, Hkv, _ = k_bits.shape
+    dQ = np.zeros((total_q, Hq, d))
+    dK = np.zeros((total_k, Hkv, d))
+    dV = np.zeros((total_k, Hkv, d))
+    for s in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[s]), int(cu_q[s + 1]), int(cu_k[s]), int(cu_k[s + 1])
+        if q1 == q0 or k1 == k0:
+            continue  # no query or no key: every gradient of the sequence is 0
+        seq = lambda x, a, b: np.ascontiguousarray(x[a:b].transpose(1, 0, 2))[None]  # noqa: E731
+        gq, gk, gv = attention_bwd_fp64(seq(q_bits, q0, q1), seq(k_bits, k0, k1), seq(v_bits, k0, k1),
+                                        seq(do_bits, q0, q1), causal, scale)
+        dQ[q0:q1] = gq[0].transpose(1, 0, 2)
+        dK[k0:k1] = gk[0].transpose(1, 0, 2)
+        dV[k0:k1] = gv[0].transpose(1, 0, 2)
+    return dQ, dK, dV

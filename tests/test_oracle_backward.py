@@ -98,3 +98,61 @@ def test_row_blocked_head_matches_whole_matrix(block_rows):
             assert np.max(np.abs(blk["O"] - O[0, 0, blk["i0"]:blk["i1"]])) < 1e-13
             assert np.max(np.abs(blk["LSE"] - L[0, 0, blk["i0"]:blk["i1"]])) < 1e-13
     assert np.max(np.abs(gK - dK[0, 0])) < 1e-13 and np.max(np.abs(gV - dV[0, 0])) < 1e-13
+
+
+def _packed(lens_q, lens_k, Hq, Hkv, d, seed):
+    g = torch.Generator().manual_seed(seed)
+    tq, tk = sum(lens_q), sum(lens_k)
+    q = torch.randn((tq, Hq, d), generator=g).to(torch.bfloat16)
+    k = torch.randn((tk, Hkv, d), generator=g).to(torch.bfloat16)
+    v = torch.randn((tk, Hkv, d), generator=g).to(torch.bfloat16)
+    do = torch.randn((tq, Hq, d), generator=g).to(torch.bfloat16)
+    cq = np.concatenate([[0], np.cumsum(lens_q)]).astype(np.int64)
+    ck = np.concatenate([[0], np.cumsum(lens_k)]).astype(np.int64)
+    return bf16_bits(q), bf16_bits(k), bf16_bits(v), bf16_bits(do), cq, ck
+
+
+def test_varlen_backward_equal_lengths_is_dense_backward():
+    B, H, N, d = 3, 2, 20, 8
+    qb, kb, vb, dob = _inputs(B, H, H, N, N, d, seed=40)
+    dQ, dK, dV = oracle.attention_bwd_fp64(qb, kb, vb, dob, True, 0.3)
+    pack = lambda x: np.ascontiguousarray(x.transpose(0, 2, 1, 3).reshape(B * N, H, d))  # noqa: E731
+    cu = np.arange(0, (B + 1) * N, N)
+    gq, gk, gv = oracle.backward.attention_varlen_bwd_fp64(pack(qb), pack(kb), pack(vb), pack(dob),
+                                                           cu, cu, True, 0.3)
+    assert np.array_equal(gq, pack(dQ)) and np.array_equal(gk, pack(dK)) and np.array_equal(gv, pack(dV))
+
+
+def test_varlen_backward_finite_differences():
+    """Central differences of <O, dO> through the packed forward oracle, with
+    unequal lengths, a prefix of keys (cache) and an empty key set."""
+    qb, kb, vb, dob, cq, ck = _packed([3, 2, 4], [5, 0, 4], 2, 1, 4, seed=41)
+    scale = 0.5
+    dQ, dK, dV = oracle.backward.attention_varlen_bwd_fp64(qb, kb, vb, dob, cq, ck, True, scale)
+    w = oracle.widen_bf16
+    q, k, v, do = w(qb), w(kb), w(vb), w(dob)
+
+    def loss(q_, k_, v_):
+        # <O, dO> with O from the definition on float64 inputs, sequence by
+        # sequence (the packed forward oracle takes bf16 bits, which a
+        # perturbed input is not)
+        total = 0.0
+        for s in range(len(cq) - 1):
+            a, b, c, e = cq[s], cq[s + 1], ck[s], ck[s + 1]
+            if b == a:
+                continue
+            t = lambda x, i, j: x[i:j].transpose(1, 0, 2)[None]  # noqa: E731
+            O, _ = oracle.attention_f64(t(q_, a, b), t(k_, c, e), t(v_, c, e), True, scale)
+            total += float((O[0].transpose(1, 0, 2) * do[a:b]).sum())
+        return total
+    eps = 1e-6
+    for x, g in ((q, dQ), (k, dK), (v, dV)):
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            fd = (loss(*[xp if x is a else a for a in (q, k, v)]) -
+                  loss(*[xm if x is a else a for a in (q, k, v)])) / (2 * eps)
+            assert abs(fd - g[idx]) < 1e-7
