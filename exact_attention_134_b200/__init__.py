@@ -55,6 +55,8 @@ _SIGNATURES = {
     "attn_q8_workspace_offsets": (_c_int, [_c_int] * 6 + [ctypes.POINTER(_sz)]),
     "attn_bwd_workspace_size": (_sz, [_c_int] * 6),
     "attn_bwd": (_c_int, [_vp] * 9 + [_c_int] * 7 + [_c_float, _vp, _sz, _vp]),
+    "attn_bwd_varlen_workspace_size": (_sz, [_c_int] * 4),
+    "attn_bwd_varlen": (_c_int, [_vp] * 11 + [_c_int] * 9 + [_c_float, _vp, _sz, _vp]),
     "attn_selftest_wait_timeout": (_c_int, [_c_int, _vp]),
     "attn_get_status": (_c_int, [_vp]),
     "attn_get_status_ex": (_c_int, [_vp, ctypes.POINTER(_c_int)]),
@@ -204,6 +206,50 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                         _stream_handle(q.device))
     _check(st, "attn_bwd")
+    return dq, dk, dv
+
+
+def attn_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                    max_seqlen_k: int, causal: bool = False, scale: float | None = None,
+                    workspace=None, dq=None, dk=None, dv=None):
+    """Gradients of attn_fwd_varlen on the GPU (packed sequences).
+
+    q, o, dout: bf16 cuda [total_q, Hq, d]; k, v: [total_k, Hkv, d]; lse: fp32
+    [Hq, total_q] (the varlen forward's); cu_seqlens_*: int32 cuda
+    [num_seqs + 1]. Returns (dq, dk, dv) in the layouts of q, k, v.
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor [total, H, d]")
+    for name, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.dim() != 1:
+            raise ValueError(f"{name} must be a contiguous int32 CUDA vector")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both hold num_seqs + 1 offsets")
+    total_q, Hq, d = q.shape
+    total_k, Hkv, dk_ = k.shape
+    if tuple(v.shape) != tuple(k.shape) or dk_ != d or tuple(o.shape) != tuple(q.shape) or \
+            tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch")
+    if lse.dtype != torch.float32 or not lse.is_cuda or tuple(lse.shape) != (Hq, total_q):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [Hq, total_q]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    n = cu_seqlens_q.numel() - 1
+    if workspace is None:
+        need = int(lib().attn_bwd_varlen_workspace_size(n, Hq, int(max_seqlen_q), d))
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = lib().attn_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                               dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                               cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), n, int(max_seqlen_q),
+                               int(max_seqlen_k), total_q, total_k, Hq, Hkv, d, int(bool(causal)),
+                               float(scale), workspace.data_ptr(),
+                               workspace.numel() * workspace.element_size(), _stream_handle(q.device))
+    _check(st, "attn_bwd_varlen")
     return dq, dk, dv
 
 

@@ -352,32 +352,44 @@ BwdLayout bwd_layout(int B, int Hq, int Nq, int d) {
   return L;
 }
 
+// Backward for dense tensors (cu_q == nullptr: B batch entries, Nq / Nkv rows
+// each) or packed sequences (B = sequences, Nq / Nkv = total rows, rows of a
+// sequence up to max_q / max_k).
 attn_status_t run_bwd(const void* q, const void* k, const void* v, const void* o,
-                      const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
-                      int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
-                      void* workspace, cudaStream_t stream) {
+                      const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                      const int* cu_q, const int* cu_k, int B, int Hq, int Hkv, int Nq, int Nkv,
+                      int max_q, int max_k, int d, int causal, float scale, void* workspace,
+                      cudaStream_t stream) {
   int* status = device_status_ptr();
   if (!status) return ATTN_ERR_CUDA;
-  const BwdLayout W = bwd_layout(B, Hq, Nq, d);
+  const bool vl = cu_q != nullptr;
+  const BwdLayout W = bwd_layout(B, Hq, max_q, d);
   char* w = static_cast<char*>(workspace);
   attn_sm100::BwdLaunch L;
   std::memset(static_cast<void*>(&L), 0, sizeof(L));
-  if (!make_map(&L.tq, q, d, Nq, (long long)B * Hq) || !make_map(&L.tk, k, d, Nkv, (long long)B * Hkv) ||
-      !make_map(&L.tv, v, d, Nkv, (long long)B * Hkv) ||
-      !make_map(&L.tdo, dout, d, Nq, (long long)B * Hq))
-    return ATTN_ERR_CUDA;
-  const int nq_pad = (Nq + 127) / 128 * 128;
+  const bool maps_ok =
+      vl ? make_map_packed(&L.tq, q, d, Hq, Nq) && make_map_packed(&L.tk, k, d, Hkv, Nkv) &&
+               make_map_packed(&L.tv, v, d, Hkv, Nkv) && make_map_packed(&L.tdo, dout, d, Hq, Nq)
+         : make_map(&L.tq, q, d, Nq, (long long)B * Hq) &&
+               make_map(&L.tk, k, d, Nkv, (long long)B * Hkv) &&
+               make_map(&L.tv, v, d, Nkv, (long long)B * Hkv) &&
+               make_map(&L.tdo, dout, d, Nq, (long long)B * Hq);
+  if (!maps_ok) return ATTN_ERR_CUDA;
+  const int nq_pad = (max_q + 127) / 128 * 128;
   float* acc = reinterpret_cast<float*>(w + W.acc);
   float* lse2 = reinterpret_cast<float*>(w + W.lse2);
   float* dvec = reinterpret_cast<float*>(w + W.dvec);
   L.B = B;
+  L.max_kv = max_k;
   L.pre.o = o;
   L.pre.dout = dout;
   L.pre.lse = lse;
   L.pre.dvec = dvec;
   L.pre.lse2 = lse2;
   L.pre.dq_acc = acc;
+  L.pre.cu_q = cu_q;
   L.pre.Nq = Nq;
+  L.pre.Hq = Hq;
   L.pre.nq_pad = nq_pad;
   attn_sm100::BwdParams& p = L.main;
   p.dk = dk;
@@ -386,6 +398,8 @@ attn_status_t run_bwd(const void* q, const void* k, const void* v, const void* o
   p.lse2 = lse2;
   p.dvec = dvec;
   p.status = status;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
   p.Nq = Nq;
   p.Nkv = Nkv;
   p.Hq = Hq;
@@ -397,7 +411,9 @@ attn_status_t run_bwd(const void* q, const void* k, const void* v, const void* o
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
   L.post.dq_acc = acc;
   L.post.dq = dq;
+  L.post.cu_q = cu_q;
   L.post.Nq = Nq;
+  L.post.Hq = Hq;
   L.post.nq_pad = nq_pad;
   L.post.scale = scale;
   return cuda_status(attn_sm100::launch_bwd(L, d, stream));
@@ -595,13 +611,12 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, false);
   if (s != ATTN_OK) return s;
   if (!dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
-  if ((long long)B * Hq > 65535) return ATTN_ERR_UNSUPPORTED;  // grid y of the row kernels
   if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return ATTN_ERR_ALIGNMENT;
   if (!workspace || !aligned16(workspace) ||
       workspace_bytes < bwd_layout(B, Hq, Nq, d).total)
     return ATTN_ERR_WORKSPACE;
-  return run_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nkv, d, causal, scale,
-                 workspace, static_cast<cudaStream_t>(stream));
+  return run_bwd(q, k, v, o, lse, dout, dq, dk, dv, nullptr, nullptr, B, Hq, Hkv, Nq, Nkv, Nq, Nkv, d,
+                 causal, scale, workspace, static_cast<cudaStream_t>(stream));
 }
 
 attn_status_t attn_selftest_wait_timeout(int budget_us, void* stream) {
@@ -611,6 +626,35 @@ attn_status_t attn_selftest_wait_timeout(int budget_us, void* stream) {
   selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       status, 1000ull * (unsigned long long)budget_us);
   return cuda_status(cudaGetLastError());
+}
+
+size_t attn_bwd_varlen_workspace_size(int num_seqs, int Hq, int max_seqlen_q, int d) {
+  if (num_seqs <= 0 || Hq <= 0 || max_seqlen_q <= 0 || d <= 0) return 0;
+  return bwd_layout(num_seqs, Hq, max_seqlen_q, d).total;
+}
+
+attn_status_t attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                              const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                              const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                              int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int Hq,
+                              int Hkv, int d, int causal, float scale, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!cu_seqlens_q || !cu_seqlens_k) return ATTN_ERR_INVALID_ARG;
+  if (num_seqs <= 0 || max_seqlen_q <= 0 || max_seqlen_k <= 0) return ATTN_ERR_INVALID_ARG;
+  // the dense checks with B = 1 cover pointers, sizes, heads, scale, d and alignment
+  attn_status_t s = check_args(q, k, v, o, lse, 1, Hq, Hkv, total_q, total_k, d, causal, scale, false);
+  if (s != ATTN_OK) return s;
+  if (!dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return ATTN_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) | reinterpret_cast<uintptr_t>(cu_seqlens_k)) & 3u)
+    return ATTN_ERR_ALIGNMENT;
+  if (num_seqs > 65535) return ATTN_ERR_UNSUPPORTED;
+  if (!workspace || !aligned16(workspace) ||
+      workspace_bytes < bwd_layout(num_seqs, Hq, max_seqlen_q, d).total)
+    return ATTN_ERR_WORKSPACE;
+  return run_bwd(q, k, v, o, lse, dout, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, num_seqs, Hq, Hkv,
+                 total_q, total_k, max_seqlen_q, max_seqlen_k, d, causal, scale, workspace,
+                 static_cast<cudaStream_t>(stream));
 }
 
 attn_status_t attn_get_status_ex(void* stream, int* where) {

@@ -180,7 +180,12 @@ __device__ __forceinline__ void store_row(uint32_t t_row, float mul, uint16_t* d
   }
 }
 
-template <int D>
+// VL = false: dense [B, H, N, d] tensors, grid z = batch entry.
+// VL = true : packed variable-length sequences [total, H, d], grid z =
+//             sequence; rows past a sequence's end (the next sequence's) are
+//             loaded but contribute nothing: their keys are masked and their
+//             queries carry LSE_2 = +inf (P = dS = 0).
+template <int D, bool VL>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -196,14 +201,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- work unit: 128 keys of one (batch, kv head)
   const int kb = blockIdx.x;
   const int hk = blockIdx.y;
-  const int b = blockIdx.z;
+  const int b = blockIdx.z;  // batch entry, or sequence (VL)
   const int G = p.Hq / p.Hkv;
   const int k0 = kb * kBK;
-  const int bh_kv = b * p.Hkv + hk;
+  int Lq = p.Nq, Lk = p.Nkv, q_start = 0, k_start = 0;
+  if (VL) {
+    q_start = min(max(p.cu_q[b], 0), p.Nq);
+    // rows past max_seqlen_q (nq_pad) are not computed: they have no
+    // accumulator rows
+    Lq = min(min(max(p.cu_q[b + 1], q_start), p.Nq) - q_start, p.nq_pad);
+    k_start = min(max(p.cu_k[b], 0), p.Nkv);
+    Lk = min(max(p.cu_k[b + 1], k_start), p.Nkv) - k_start;
+    if (k0 >= Lk) return;  // this sequence has fewer keys (the whole CTA leaves)
+  }
+  // row of key k0 + r in dK / dV, and TMA coordinates of K/V and Q/dO tiles
+  auto kv_row_off = [&](int r) -> size_t {
+    return VL ? ((size_t)(k_start + k0 + r) * p.Hkv + hk) * D
+              : ((size_t)(b * p.Hkv + hk) * p.Nkv + k0 + r) * D;
+  };
   // causal mask aligned to the bottom right: key j is visible to query i iff
-  // j <= i + (Nkv - Nq). The first query block with a visible pair:
-  const int diag = p.causal ? p.Nkv - p.Nq : 0;
-  const int nqb = (p.Nq + kBQ - 1) / kBQ;
+  // j <= i + (Lk - Lq). The first query block with a visible pair:
+  const int diag = p.causal ? Lk - Lq : 0;
+  const int nqb = (Lq + kBQ - 1) / kBQ;
   int j_begin = 0;
   if (p.causal) j_begin = max(0, k0 - diag) / kBQ;
   const int n_iter = max(0, nqb - j_begin) * G;
@@ -216,8 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       return;
     }
     for (int r = threadIdx.x; r < kBK; r += kThreads) {
-      if (k0 + r >= p.Nkv) break;
-      const size_t off = ((size_t)bh_kv * p.Nkv + k0 + r) * D;
+      if (k0 + r >= Lk) break;
+      const size_t off = kv_row_off(r);
       uint4* dk = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dk) + off);
       uint4* dv = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dv) + off);
       for (int i = 0; i < D / 8; ++i) dk[i] = dv[i] = make_uint4(0, 0, 0, 0);
@@ -284,8 +303,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       mbar_arrive_expect_tx(bar(Bars::kKV), 2 * C::kTileBytes);
       for (int bx = 0; bx < C::kBoxes; ++bx) {
-        tma_load_3d(sK + bx * C::kBoxBytes, &tm_k, bar(Bars::kKV), bx * 64, k0, bh_kv);
-        tma_load_3d(sV + bx * C::kBoxBytes, &tm_v, bar(Bars::kKV), bx * 64, k0, bh_kv);
+        const int c1 = VL ? hk : k0, c2 = VL ? k_start + k0 : b * p.Hkv + hk;
+        tma_load_3d(sK + bx * C::kBoxBytes, &tm_k, bar(Bars::kKV), bx * 64, c1, c2);
+        tma_load_3d(sV + bx * C::kBoxBytes, &tm_v, bar(Bars::kKV), bx * 64, c1, c2);
       }
     }
     int half = 0;  // 0: Q + LSE_2 of query block it; 1: its dO + D
@@ -296,12 +316,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       if (lane == 0) {
         const int q0 = q_block(it) * kBQ;
-        const int bh_q = b * p.Hq + q_head(it);
+        const int h = q_head(it);
+        const int bh_q = b * p.Hq + h;  // (batch or sequence, head): row of LSE_2 / D
         const uint32_t fb = bar((half ? Bars::kFullDO : Bars::kFull) + s);
         mbar_arrive_expect_tx(fb, C::kHalfBytes);
         for (int bx = 0; bx < C::kBoxes; ++bx)
           tma_load_3d((half ? sDO(s) : sQ(s)) + bx * C::kBoxBytes, half ? &tm_do : &tm_q, fb, bx * 64,
-                      q0, bh_q);
+                      VL ? h : q0, VL ? q_start + q0 : bh_q);
         const size_t voff = (size_t)bh_q * p.nq_pad + q0;
         bulk_load(base + C::kOffVec + (2 * half + s) * kBQ * 4, (half ? p.dvec : p.lse2) + voff,
                   kBQ * 4, fb);
@@ -400,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kr = threadIdx.x;  // key row within the block == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(warp << 5) << 16;
     const uint32_t tS = tmem + C::kColS + lane_off, tDP = tmem + C::kColDP + lane_off;
-    const bool key_valid = k0 + kr < p.Nkv;
+    const bool key_valid = k0 + kr < Lk;
     const float sl2 = p.scale_log2;
     uint8_t* const ds_row = base_ptr + C::kOffDS + kr * 128;
     bool ok = true;
@@ -485,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) ok = warp_all(bounded_wait(bar(Bars::kAcc), 0, abort_flag, budget));
     if (ok) {
       tc_fence_after();
-      uint16_t* dst = static_cast<uint16_t*>(p.dk) + ((size_t)bh_kv * p.Nkv + (key_valid ? k0 + kr : 0)) * D;
+      uint16_t* dst = static_cast<uint16_t*>(p.dk) + kv_row_off(key_valid ? kr : 0);
       store_row<D>(tmem + C::kColDK + lane_off, p.scale, dst, key_valid);
     } else if (lane == 0) {
       flag_abort(abort_flag, p.status, 0x300 | (it << 12));
@@ -552,8 +573,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       const int kr = wq * 32 + lane;
-      const bool key_valid = k0 + kr < p.Nkv;
-      uint16_t* dst = static_cast<uint16_t*>(p.dv) + ((size_t)bh_kv * p.Nkv + (key_valid ? k0 + kr : 0)) * D;
+      const bool key_valid = k0 + kr < Lk;
+      uint16_t* dst = static_cast<uint16_t*>(p.dv) + kv_row_off(key_valid ? kr : 0);
       store_row<D>(tmem + C::kColDV + lane_off, 1.0f, dst, key_valid);
     } else if (lane == 0) {
       flag_abort(abort_flag, p.status, 0x500 | (it << 12));
@@ -569,18 +590,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// D_i = sum_c dO_ic O_ic (fp32), LSE_2 = LSE * log2(e) (+inf for rows past Nq
+// Rows of one (batch entry or sequence, head): their count, and the offsets of
+// row r in the [.., H, d]-shaped tensors and in LSE ([B, H, N] dense,
+// [H, total] packed).
+template <int D, bool VL>
+struct RowMap {
+  int L, start;
+  size_t head_base;  // dense: (s * H + h) * N
+  int h, H;
+  __device__ RowMap(const int* cu, int s, int h_, int H_, int N) : h(h_), H(H_) {
+    if (VL) {
+      start = min(max(cu[s], 0), N);
+      L = min(max(cu[s + 1], start), N) - start;
+      head_base = 0;
+    } else {
+      start = 0;
+      L = N;
+      head_base = ((size_t)s * H + h_) * N;
+    }
+  }
+  __device__ size_t row(int r) const {  // element offset of row r, column 0
+    return VL ? ((size_t)(start + r) * H + h) * D : (head_base + r) * D;
+  }
+  __device__ size_t lse(int r, int N) const {
+    return VL ? (size_t)h * N + start + r : head_base + r;
+  }
+};
+
+// D_i = sum_c dO_ic O_ic (fp32), LSE_2 = LSE * log2(e) (+inf for padding rows
 // and for rows that saw no key, so their P is 0), and the dQ accumulator rows
-// zeroed. Block = 256 threads = 32 rows x 8 threads per row.
-template <int D>
+// zeroed. Grid (nq_pad / 32, Hq, batch entries or sequences); block = 256
+// threads = 32 rows x 8 threads per row.
+template <int D, bool VL>
 __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const BwdPreParams p) {
-  const int g = blockIdx.x;           // 32-row group
-  const int bh = blockIdx.y;
+  const int g = blockIdx.x;  // 32-row group
+  const int h = blockIdx.y, sq = blockIdx.z;
+  const RowMap<D, VL> m(p.cu_q, sq, h, p.Hq, p.Nq);
+  const size_t bh = (size_t)sq * p.Hq + h;
   const int r = g * 32 + (threadIdx.x >> 3);
   const int part = threadIdx.x & 7;   // D/8 columns each
   float acc = 0.0f;
-  if (r < p.Nq) {
-    const size_t row = ((size_t)bh * p.Nq + r) * D + part * (D / 8);
+  if (r < m.L) {
+    const size_t row = m.row(r) + part * (D / 8);
     const uint4* o = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.o) + row);
     const uint4* g4 = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + row);
 #pragma unroll
@@ -598,31 +649,34 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const BwdPreParams p)
   acc += __shfl_xor_sync(0xffffffffu, acc, 2);
   acc += __shfl_xor_sync(0xffffffffu, acc, 4);
   if (part == 0) {
-    const size_t v = (size_t)bh * p.nq_pad + r;
+    const size_t v = bh * p.nq_pad + r;
     p.dvec[v] = acc;
     float l2 = INFINITY;
-    if (r < p.Nq) {
-      const float l = p.lse[(size_t)bh * p.Nq + r];
+    if (r < m.L) {
+      const float l = p.lse[m.lse(r, p.Nq)];
       if (l != -INFINITY) l2 = l * 1.4426950408889634f;
     }
     p.lse2[v] = l2;
   }
-  // zero the accumulator's floats [32 D g, 32 D (g + 1)) of this head (the
-  // groups of a head together cover its nq_pad * D floats, whatever the layout)
-  float4* acc_rows = reinterpret_cast<float4*>(p.dq_acc + ((size_t)bh * p.nq_pad + g * 32) * D);
+  // zero the accumulator's floats [32 D g, 32 D (g + 1)) of this (sequence,
+  // head) (the groups together cover its nq_pad * D floats, whatever the layout)
+  float4* acc_rows = reinterpret_cast<float4*>(p.dq_acc + (bh * p.nq_pad + g * 32) * D);
   for (int i = threadIdx.x; i < 8 * D; i += 256) acc_rows[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // dQ = bf16(scale * accumulator), through a shared-memory transpose so both
 // the accumulator reads and the dQ row writes are contiguous. The accumulator
 // holds each 128-row block as [d/4][128 rows][4]; a CTA converts 32 rows.
-template <int D>
+template <int D, bool VL>
 __global__ void __launch_bounds__(256) attn_bwd_post_kernel(const BwdPostParams p) {
   constexpr int kPitch = D + 8;  // bf16 elements per staged row (breaks bank conflicts)
   __shared__ __align__(16) uint16_t tile[32 * kPitch];
   const int g = blockIdx.x;
-  const int bh = blockIdx.y;
-  const float4* src = reinterpret_cast<const float4*>(p.dq_acc + ((size_t)bh * p.nq_pad + (g >> 2) * kBQ) * D) +
+  const int h = blockIdx.y, sq = blockIdx.z;
+  const RowMap<D, VL> m(p.cu_q, sq, h, p.Hq, p.Nq);
+  const size_t bh = (size_t)sq * p.Hq + h;
+  if (g * 32 >= m.L) return;  // nothing of this sequence in these rows
+  const float4* src = reinterpret_cast<const float4*>(p.dq_acc + (bh * p.nq_pad + (g >> 2) * kBQ) * D) +
                       (g & 3) * 32;
   for (int i = threadIdx.x; i < 8 * D; i += 256) {
     const int c4 = i >> 5, row = i & 31;
@@ -636,35 +690,36 @@ __global__ void __launch_bounds__(256) attn_bwd_post_kernel(const BwdPostParams 
   for (int i = threadIdx.x; i < 32 * (D / 8); i += 256) {
     const int row = i / (D / 8), c8 = i % (D / 8);
     const int r = g * 32 + row;
-    if (r < p.Nq)
-      *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dq) + ((size_t)bh * p.Nq + r) * D + 8 * c8) =
+    if (r < m.L)
+      *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dq) + m.row(r) + 8 * c8) =
           *reinterpret_cast<const uint4*>(&tile[row * kPitch + 8 * c8]);
   }
 }
 
-template <int D>
+template <int D, bool VL>
 cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
-  const int groups = L.pre.nq_pad / 32;
-  const long long bhq = (long long)L.B * L.main.Hq;
-  attn_bwd_pre_kernel<D><<<dim3(groups, (unsigned)bhq), 256, 0, stream>>>(L.pre);
+  const dim3 rows_grid(L.pre.nq_pad / 32, L.main.Hq, L.B);  // B: batch entries or sequences
+  attn_bwd_pre_kernel<D, VL><<<rows_grid, 256, 0, stream>>>(L.pre);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(attn_bwd_main_kernel<D, VL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            BwdCfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((L.main.Nkv + kBK - 1) / kBK, L.main.Hkv, L.B);
-  attn_bwd_main_kernel<D><<<grid, kThreads, BwdCfg<D>::kSmemBytes, stream>>>(L.tq, L.tk, L.tv, L.tdo,
-                                                                          L.main);
+  dim3 grid((L.max_kv + kBK - 1) / kBK, L.main.Hkv, L.B);
+  attn_bwd_main_kernel<D, VL><<<grid, kThreads, BwdCfg<D>::kSmemBytes, stream>>>(L.tq, L.tk, L.tv, L.tdo,
+                                                                              L.main);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_bwd_post_kernel<D><<<dim3(groups, (unsigned)bhq), 256, 0, stream>>>(L.post);
+  attn_bwd_post_kernel<D, VL><<<rows_grid, 256, 0, stream>>>(L.post);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_bwd(const BwdLaunch& L, int d, cudaStream_t stream) {
-  return d == 128 ? launch_bwd_d<128>(L, stream) : launch_bwd_d<64>(L, stream);
+  const bool vl = L.main.cu_q != nullptr;
+  if (d == 128) return vl ? launch_bwd_d<128, true>(L, stream) : launch_bwd_d<128, false>(L, stream);
+  return vl ? launch_bwd_d<64, true>(L, stream) : launch_bwd_d<64, false>(L, stream);
 }
 
 }  // namespace attn_sm100

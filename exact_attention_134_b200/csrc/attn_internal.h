@@ -65,11 +65,13 @@ cudaError_t launch_q8(const Q8Launch& L, int d, cudaStream_t stream);
 struct BwdParams {
   void* dk;                       // bf16 [B, Hkv, Nkv, d]
   void* dv;                       // bf16 [B, Hkv, Nkv, d]
-  float* dq_acc;                  // fp32 [B*Hq][nq_pad/128][d/4][128][4]
+  float* dq_acc;                  // fp32 [B*Hq][nq_pad/128][d/4][128][4] (packed: B = sequences)
   const float* lse2;              // fp32 [B*Hq][nq_pad]  LSE * log2(e), +inf where P must be 0
   const float* dvec;              // fp32 [B*Hq][nq_pad]  D_i = sum_c dO_ic O_ic
   int* status;
-  int Nq, Nkv, Hq, Hkv;
+  const int* cu_q;                // packed sequences: row offsets [B + 1] (else null)
+  const int* cu_k;
+  int Nq, Nkv, Hq, Hkv;           // packed: Nq / Nkv = total rows, B = sequences
   int causal;
   int nq_pad;                     // Nq rounded up to 128
   float scale;
@@ -84,13 +86,15 @@ struct BwdPreParams {
   float* dvec;
   float* lse2;
   float* dq_acc;
-  int Nq, nq_pad;
+  const int* cu_q;                // packed sequences (else null)
+  int Nq, Hq, nq_pad;
 };
 
 struct BwdPostParams {
   const float* dq_acc;
-  void* dq;                       // bf16 [B, Hq, Nq, d]
-  int Nq, nq_pad;
+  void* dq;                       // bf16 [B, Hq, Nq, d] (packed: [total_q, Hq, d])
+  const int* cu_q;
+  int Nq, Hq, nq_pad;
   float scale;
 };
 
@@ -99,7 +103,8 @@ struct BwdLaunch {
   BwdParams main;
   BwdPreParams pre;
   BwdPostParams post;
-  int B;
+  int B;                          // batch entries, or sequences
+  int max_kv;                     // Nkv, or the longest sequence's keys
 };
 
 cudaError_t launch_bwd(const BwdLaunch& L, int d, cudaStream_t stream);

@@ -232,7 +232,7 @@ ATTN_API attn_status_t attn_q8_workspace_offsets(int B, int Hq, int Hkv, int Nq,
  *   workspace      device scratch of attn_bwd_workspace_size() bytes, 16-byte
  *                  aligned, owned by the caller; holds the fp32 dQ
  *                  accumulator, D and LSE * log2(e); needs no initial value
- * d must be 64 or 128 (96: ATTN_ERR_UNSUPPORTED), B * Hq <= 65535. The dQ accumulation adds
+ * d must be 64 or 128 (96, 256: ATTN_ERR_UNSUPPORTED). The dQ accumulation adds
  * fp32 partial sums with atomics, so dQ may differ in the last bits between
  * runs; dK and dV are deterministic. Errors as attn_fwd, plus
  * ATTN_ERR_WORKSPACE for a missing, misaligned or short workspace.
@@ -243,6 +243,28 @@ ATTN_API attn_status_t attn_bwd(const void* q, const void* k, const void* v, con
                                 int B, int Hq, int Hkv, int Nq, int Nkv, int d, int causal,
                                 float scale, void* workspace, size_t workspace_bytes,
                                 void* stream);
+
+/*
+ * attn_bwd_varlen — attn_bwd for packed variable-length sequences, the
+ * gradients of attn_fwd_varlen: q, o, dout, dq [total_q, Hq, d]; k, v, dk, dv
+ * [total_k, Hkv, d]; lse fp32 [Hq, total_q] as attn_fwd_varlen writes it;
+ * cu_seqlens_q / cu_seqlens_k int32 device arrays [num_seqs + 1] (sequence s
+ * owns rows cu[s] .. cu[s+1]); max_seqlen_q / max_seqlen_k must bound every
+ * sequence's rows (they size the grid and the workspace; rows beyond them are
+ * not computed, and nothing outside the buffers is touched). Causal masks are
+ * aligned to the bottom right of each sequence. Rows of dk / dv that no
+ * query sees are written as 0. Workspace: attn_bwd_varlen_workspace_size()
+ * bytes (fp32 dQ accumulator with every sequence padded to max_seqlen_q
+ * rows, then LSE * log2(e) and D). Errors as attn_bwd and attn_fwd_varlen.
+ */
+ATTN_API size_t attn_bwd_varlen_workspace_size(int num_seqs, int Hq, int max_seqlen_q, int d);
+ATTN_API attn_status_t attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                                       const float* lse, const void* dout, void* dq, void* dk,
+                                       void* dv, const int* cu_seqlens_q,
+                                       const int* cu_seqlens_k, int num_seqs, int max_seqlen_q,
+                                       int max_seqlen_k, int total_q, int total_k, int Hq,
+                                       int Hkv, int d, int causal, float scale, void* workspace,
+                                       size_t workspace_bytes, void* stream);
 
 /*
  * attn_get_status — synchronises `stream`, returns and clears the device
