@@ -30,7 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from synthetic import (VARLEN_WORKLOADS, WORKLOADS, Workload, bf16_bits, make_dout, make_qkv,  # noqa: E402
-                       make_varlen)
+                       make_varlen, make_varlen_dout)
 
 HEADLINE = "outlier_8k_causal"
 EXTRA_BF16 = ["tiny_256_d64", "causal_2k_d128", "outlier_8k_full", "gqa_32k_d128", "gqa_32k_d64",
@@ -328,6 +328,36 @@ def bench_bwd(w: Workload, steps: int, warmup: int, world: int, rank: int, lib_m
             "l2": "inputs_larger_than_l2"}
 
 
+def bench_varlen_bwd(name: str, steps: int, warmup: int, world: int, lib_mod, peak: float):
+    """Backward of the packed variable-length workload (after one forward)."""
+    import torch
+    w = VARLEN_WORKLOADS[name]
+    q, k, v, cu = make_varlen(w)
+    do = make_varlen_dout(w)
+    qd, kd, vd, dod, cud = q.cuda(), k.cuda(), v.cuda(), do.cuda(), cu.cuda()
+    max_len = max(w.lengths())
+    o, lse = lib_mod.attn_fwd_varlen(qd, kd, vd, cud, cud, max_len, causal=w.causal)
+    need = lib_mod.lib().attn_bwd_varlen_workspace_size(w.num_seqs, w.Hq, max_len, w.d)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+
+    def step():
+        lib_mod.attn_bwd_varlen(qd, kd, vd, o, lse, dod, cud, cud, max_len, max_len, causal=w.causal,
+                                workspace=ws, dq=dq, dk=dk, dv=dv)
+
+    _barrier(world)
+    times = time_device(step, steps, max(warmup, 3))
+    _barrier(world)
+    st, where = lib_mod.get_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} at {where:#x}")
+    ms = _max_over_ranks(statistics.mean(times), world)
+    tf = world * 2.5 * w.flops / (ms * 1e-3) / 1e12
+    return {"tflops": round(tf, 1), "ms_per_step": round(ms, 4), "frac_of_bf16_peak": round(tf / world / peak, 4),
+            "flops": "2.5 x forward (five N x N x d products)", "sequences": w.num_seqs,
+            "total_tokens": int(q.shape[0]), "l2": "inputs_larger_than_l2"}
+
+
 def bench_e2e(w: Workload, steps: int, warmup: int, world: int, rank: int, lib_mod):
     """Same metric through the host-buffer entry point: every step copies the
     step's inputs from pinned host memory and reads O and LSE back."""
@@ -430,6 +460,10 @@ def run_ours(args):
             extras["backward_" + name] = bench_bwd(WORKLOADS[name], max(3, args.steps // 2), 3, world,
                                                    rank, attn, peaks["bf16"])
             torch.cuda.empty_cache()
+        extras["backward_varlen_prefill_mixed"] = bench_varlen_bwd("varlen_prefill_mixed",
+                                                                   max(3, args.steps // 2), 3, world,
+                                                                   attn, peaks["bf16"])
+        torch.cuda.empty_cache()
         wq = WORKLOADS["q8_8k_outlier"]
         full_ms, pre_ms = bench_q8(wq, max(3, args.steps // 2), 3, world, rank, attn)
         fp8_peak = 2.0 * peaks["bf16"]

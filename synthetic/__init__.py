@@ -186,3 +186,11 @@ def make_varlen(w: VarlenWorkload):
     v = torch.randn((total, w.Hkv, w.d), generator=g, dtype=torch.float32)
     cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
     return _bf16(q), _bf16(k), _bf16(v), cu
+
+
+def make_varlen_dout(w: VarlenWorkload) -> torch.Tensor:
+    """dO for the packed workload: fp32 ``randn`` [total, Hq, d] from a
+    generator seeded with ``seed + 500``, rounded to bf16."""
+    total = sum(w.lengths())
+    g = torch.Generator("cpu").manual_seed(w.seed + 500)
+    return _bf16(torch.randn((total, w.Hq, w.d), generator=g, dtype=torch.float32))
