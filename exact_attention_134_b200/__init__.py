@@ -281,6 +281,42 @@ def _autograd_fn():
     return _AUTOGRAD_FN
 
 
+_AUTOGRAD_VARLEN_FN = None
+
+
+def _autograd_varlen_fn():
+    global _AUTOGRAD_VARLEN_FN
+    if _AUTOGRAD_VARLEN_FN is None:
+        import torch
+
+        class _AttentionVarlen(torch.autograd.Function):
+            @staticmethod
+            def forward(ctx, q, k, v, cu_q, cu_k, max_q, max_k, causal, scale):
+                o, lse = attn_fwd_varlen(q, k, v, cu_q, cu_k, max_q, causal=causal, scale=scale)
+                ctx.save_for_backward(q, k, v, o, lse, cu_q, cu_k)
+                ctx.args = (max_q, max_k, causal, scale)
+                return o
+
+            @staticmethod
+            def backward(ctx, do):
+                q, k, v, o, lse, cu_q, cu_k = ctx.saved_tensors
+                max_q, max_k, causal, scale = ctx.args
+                dq, dk, dv = attn_bwd_varlen(q, k, v, o, lse, do.contiguous(), cu_q, cu_k, max_q, max_k,
+                                             causal=causal, scale=scale)
+                return dq, dk, dv, None, None, None, None, None, None
+
+        _AUTOGRAD_VARLEN_FN = _AttentionVarlen
+    return _AUTOGRAD_VARLEN_FN
+
+
+def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                     causal: bool = False, scale: float | None = None):
+    """Differentiable attention over packed variable-length sequences: forward
+    attn_fwd_varlen, backward attn_bwd_varlen (d = 64 or 128)."""
+    return _autograd_varlen_fn().apply(q, k, v, cu_seqlens_q, cu_seqlens_k, int(max_seqlen_q),
+                                       int(max_seqlen_k), causal, scale)
+
+
 def attention(q, k, v, causal: bool = False, scale: float | None = None):
     """Differentiable exact attention for training: the forward is attn_fwd
     (O only; LSE is kept for the backward), the backward attn_bwd. Same

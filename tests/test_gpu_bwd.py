@@ -313,3 +313,21 @@ def test_varlen_bwd_equal_lengths_matches_dense():
     # dK, dV: same sums in the same order; dQ: fp32 reductions in any order
     assert torch.equal(vk, pack(gk)) and torch.equal(vv, pack(gv))
     assert ((vq.float() - pack(gq).float()).abs() <= 2 * U * pack(gq).float().abs() + 1e-6).all()
+
+
+def test_autograd_varlen_matches_dense_autograd_per_sequence():
+    lens = [130, 7, 300]
+    q, k, v, w, cq, _ = _packed_case(lens, lens, 4, 2, 128, seed=77)
+    qc, kc, vc = (t.cuda().requires_grad_() for t in (q, k, v))
+    o = attn.attention_varlen(qc, kc, vc, cq.cuda(), cq.cuda(), max(lens), max(lens), causal=True)
+    (o.float() * w.cuda().float()).sum().backward()
+    for s in range(len(lens)):
+        a, b = int(cq[s]), int(cq[s + 1])
+        seq = lambda x: x[a:b].permute(1, 0, 2).unsqueeze(0).contiguous().cuda().requires_grad_()  # noqa: E731
+        qs, ks, vs = seq(q), seq(k), seq(v)
+        od = attn.attention(qs, ks, vs, causal=True)
+        (od.float() * w[a:b].permute(1, 0, 2).unsqueeze(0).cuda().float()).sum().backward()
+        back = lambda g: g[0].permute(1, 0, 2)  # noqa: E731
+        assert torch.equal(kc.grad[a:b], back(ks.grad)) and torch.equal(vc.grad[a:b], back(vs.grad))
+        assert ((qc.grad[a:b].float() - back(qs.grad).float()).abs()
+                <= 2 * U * back(qs.grad).float().abs() + 1e-6).all()
