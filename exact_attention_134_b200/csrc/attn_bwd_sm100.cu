@@ -627,6 +627,8 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const BwdPreParams p)
   const int h = blockIdx.y, sq = blockIdx.z;
   const RowMap<D, VL> m(p.cu_q, sq, h, p.Hq, p.Nq);
   const size_t bh = (size_t)sq * p.Hq + h;
+  // only the sequence's own 128-row blocks are read or reduced into
+  if (VL && g * 32 >= (m.L + kBQ - 1) / kBQ * kBQ) return;
   const int r = g * 32 + (threadIdx.x >> 3);
   const int part = threadIdx.x & 7;   // D/8 columns each
   float acc = 0.0f;
