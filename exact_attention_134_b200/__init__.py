@@ -312,7 +312,7 @@ def _autograd_varlen_fn():
 def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
                      causal: bool = False, scale: float | None = None):
     """Differentiable attention over packed variable-length sequences: forward
-    attn_fwd_varlen, backward attn_bwd_varlen (d = 64 or 128)."""
+    attn_fwd_varlen, backward attn_bwd_varlen (d = 64, 96 or 128)."""
     return _autograd_varlen_fn().apply(q, k, v, cu_seqlens_q, cu_seqlens_k, int(max_seqlen_q),
                                        int(max_seqlen_k), causal, scale)
 
@@ -320,7 +320,7 @@ def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max
 def attention(q, k, v, causal: bool = False, scale: float | None = None):
     """Differentiable exact attention for training: the forward is attn_fwd
     (O only; LSE is kept for the backward), the backward attn_bwd. Same
-    tensors and head dims as attn_bwd (d = 64 or 128)."""
+    tensors and head dims as attn_bwd (d = 64, 96 or 128)."""
     return _autograd_fn().apply(q, k, v, causal, scale)
 
 

@@ -62,7 +62,7 @@ int* device_status_ptr() {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // d = 96 is supported by the bf16 kernels only (allow96 = false for the 8-bit
-// paths and the backward); d = 256 by the dense bf16 forward only (allow256).
+// paths); d = 256 by the dense bf16 forward only (allow256).
 attn_status_t check_args(const void* q, const void* k, const void* v, const void* o,
                          const void* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
                          int causal, float scale, bool allow96 = true, bool allow256 = false) {
@@ -608,7 +608,7 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
                        const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
                        int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
                        void* workspace, size_t workspace_bytes, void* stream) {
-  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, false);
+  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
   if (s != ATTN_OK) return s;
   if (!dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return ATTN_ERR_ALIGNMENT;
@@ -642,7 +642,7 @@ attn_status_t attn_bwd_varlen(const void* q, const void* k, const void* v, const
   if (!cu_seqlens_q || !cu_seqlens_k) return ATTN_ERR_INVALID_ARG;
   if (num_seqs <= 0 || max_seqlen_q <= 0 || max_seqlen_k <= 0) return ATTN_ERR_INVALID_ARG;
   // the dense checks with B = 1 cover pointers, sizes, heads, scale, d and alignment
-  attn_status_t s = check_args(q, k, v, o, lse, 1, Hq, Hkv, total_q, total_k, d, causal, scale, false);
+  attn_status_t s = check_args(q, k, v, o, lse, 1, Hq, Hkv, total_q, total_k, d, causal, scale);
   if (s != ATTN_OK) return s;
   if (!dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return ATTN_ERR_ALIGNMENT;

@@ -71,17 +71,26 @@ constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
 constexpr int kMaxSmem = 232448;  // 227 KB opt-in limit per CTA
 
+// Q, K, V, dO tiles: 128 rows x kBoxCols bf16 per TMA box; d = 64 / 128 use
+// 64-column boxes with the 128-byte swizzle, d = 96 three 32-column boxes with
+// the 64-byte swizzle (the descriptors below describe the same layouts). The
+// dS tile always uses 64-column boxes with the 128-byte swizzle.
 template <int D>
 struct BwdCfg {
   static constexpr int kTileBytes = 128 * D * 2;  // a 128-row bf16 tile
-  static constexpr int kBoxBytes = 128 * 128;      // 128 rows x 64 bf16 columns (128-byte swizzle)
-  static constexpr int kBoxes = D / 64;
+  static constexpr int kBoxCols = (D == 96) ? 32 : 64;
+  static constexpr int kRowBytes = kBoxCols * 2;   // swizzle width (64 or 128 B)
+  static constexpr int kBoxBytes = 128 * kRowBytes;
+  static constexpr int kBoxes = D / kBoxCols;
+  static constexpr int kAtomBytes = 8 * kRowBytes; // 8-row swizzle atom
+  static constexpr int kDSBoxBytes = 128 * 128;    // dS^T tile box: 128 keys x 64 queries
+  static_assert(kTileBytes % 1024 == 0, "tiles must keep the 1024-byte swizzle alignment");
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
   static constexpr int kOffQ = 2 * kTileBytes;     // + stage * 2 * kTileBytes
   static constexpr int kOffDO = 3 * kTileBytes;    // + stage * 2 * kTileBytes
   static constexpr int kOffDS = 6 * kTileBytes;    // dS^T tile: 128 keys x 128 queries bf16
-  static constexpr int kOffVec = kOffDS + 2 * kBoxBytes;  // LSE_2[2][128], D[2][128] (fp32)
+  static constexpr int kOffVec = kOffDS + 2 * kDSBoxBytes;  // LSE_2[2][128], D[2][128] (fp32)
   static constexpr int kOffBar = kOffVec + 4 * kBQ * 4;
   static constexpr int kBytes = kOffBar + 128;
   // dynamic shared memory is requested with up to 1 KB of slack for aligning
@@ -123,12 +132,14 @@ __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu
 // D[128 x 128] = A[128 x d] . B[128 x d]^T, both K-major tiles as TMA writes them.
 template <int D>
 __device__ __forceinline__ void issue_ss_k(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+  using C = BwdCfg<D>;
   constexpr uint32_t idesc = idesc_bf16_f32(kBK, kBQ, 0);
+  constexpr int kSteps = C::kBoxCols / 16;  // 16-column MMA steps per box
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk / 4) * BwdCfg<D>::kBoxBytes + (kk % 4) * 32;
-    mma_bf16_ss(d_tmem, smem_desc_sw128(a_smem + off, 16, 1024),
-                smem_desc_sw128(b_smem + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+    const uint32_t off = (kk / kSteps) * C::kBoxBytes + (kk % kSteps) * 32;
+    mma_bf16_ss(d_tmem, smem_desc_sw(a_smem + off, 16, C::kAtomBytes, C::kRowBytes),
+                smem_desc_sw(b_smem + off, 16, C::kAtomBytes, C::kRowBytes), idesc, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -136,10 +147,11 @@ __device__ __forceinline__ void issue_ss_k(uint32_t d_tmem, uint32_t a_smem, uin
 template <int D>
 __device__ __forceinline__ void issue_ts_mn(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
                                             bool accumulate) {
+  using C = BwdCfg<D>;
   constexpr uint32_t idesc = idesc_bf16_f32(kBK, D, 1);
 #pragma unroll
   for (int kk = 0; kk < kBQ / 16; ++kk) {
-    const uint64_t b = smem_desc_sw128(b_smem + kk * 16 * 128, BwdCfg<D>::kBoxBytes, 1024);
+    const uint64_t b = smem_desc_sw(b_smem + kk * 16 * C::kRowBytes, C::kBoxBytes, C::kAtomBytes, C::kRowBytes);
     mma_bf16_ts(d_tmem, a_tmem + kk * 8, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
@@ -148,11 +160,12 @@ __device__ __forceinline__ void issue_ts_mn(uint32_t d_tmem, uint32_t a_tmem, ui
 // keys, columns = queries) is read as an MN-major A, the K tile as an MN-major B.
 template <int D>
 __device__ __forceinline__ void issue_dq(uint32_t d_tmem, uint32_t ds_smem, uint32_t k_smem) {
+  using C = BwdCfg<D>;
   constexpr uint32_t idesc = idesc_bf16_f32_major(kBQ, D, 1, 1);
 #pragma unroll
   for (int kk = 0; kk < kBK / 16; ++kk) {
-    const uint64_t a = smem_desc_sw128(ds_smem + kk * 16 * 128, BwdCfg<D>::kBoxBytes, 1024);
-    const uint64_t b = smem_desc_sw128(k_smem + kk * 16 * 128, BwdCfg<D>::kBoxBytes, 1024);
+    const uint64_t a = smem_desc_sw128(ds_smem + kk * 16 * 128, C::kDSBoxBytes, 1024);
+    const uint64_t b = smem_desc_sw(k_smem + kk * 16 * C::kRowBytes, C::kBoxBytes, C::kAtomBytes, C::kRowBytes);
     mma_bf16_ss(d_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
   }
 }
@@ -304,8 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(bar(Bars::kKV), 2 * C::kTileBytes);
       for (int bx = 0; bx < C::kBoxes; ++bx) {
         const int c1 = VL ? hk : k0, c2 = VL ? k_start + k0 : b * p.Hkv + hk;
-        tma_load_3d(sK + bx * C::kBoxBytes, &tm_k, bar(Bars::kKV), bx * 64, c1, c2);
-        tma_load_3d(sV + bx * C::kBoxBytes, &tm_v, bar(Bars::kKV), bx * 64, c1, c2);
+        tma_load_3d(sK + bx * C::kBoxBytes, &tm_k, bar(Bars::kKV), bx * C::kBoxCols, c1, c2);
+        tma_load_3d(sV + bx * C::kBoxBytes, &tm_v, bar(Bars::kKV), bx * C::kBoxCols, c1, c2);
       }
     }
     int half = 0;  // 0: Q + LSE_2 of query block it; 1: its dO + D
@@ -321,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t fb = bar((half ? Bars::kFullDO : Bars::kFull) + s);
         mbar_arrive_expect_tx(fb, C::kHalfBytes);
         for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_load_3d((half ? sDO(s) : sQ(s)) + bx * C::kBoxBytes, half ? &tm_do : &tm_q, fb, bx * 64,
+          tma_load_3d((half ? sDO(s) : sQ(s)) + bx * C::kBoxBytes, half ? &tm_do : &tm_q, fb, bx * C::kBoxCols,
                       VL ? h : q0, VL ? q_start + q0 : bh_q);
         const size_t voff = (size_t)bh_q * p.nq_pad + q0;
         bulk_load(base + C::kOffVec + (2 * half + s) * kBQ * 4, (half ? p.dvec : p.lse2) + voff,
@@ -494,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int ch = (c & 1) * 4 + q;
-          *reinterpret_cast<uint4*>(ds_row + (c >> 1) * C::kBoxBytes + ((ch ^ (kr & 7)) << 4)) =
+          *reinterpret_cast<uint4*>(ds_row + (c >> 1) * C::kDSBoxBytes + ((ch ^ (kr & 7)) << 4)) =
               make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         }
       }
@@ -633,15 +646,17 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const BwdPreParams p)
   const int part = threadIdx.x & 7;   // D/8 columns each
   float acc = 0.0f;
   if (r < m.L) {
+    // D/8 columns per thread, read 4 at a time (8-byte loads: at d = 96 a
+    // thread's 12 columns start at a multiple of 24 bytes)
     const size_t row = m.row(r) + part * (D / 8);
-    const uint4* o = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.o) + row);
-    const uint4* g4 = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + row);
+    const uint2* o = reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.o) + row);
+    const uint2* g2 = reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.dout) + row);
 #pragma unroll
-    for (int i = 0; i < D / 64; ++i) {
-      const uint4 a = o[i], c = g4[i];
-      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
+    for (int i = 0; i < D / 32; ++i) {
+      const uint2 a = o[i], c = g2[i];
+      const uint32_t aw[2] = {a.x, a.y}, cw[2] = {c.x, c.y};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < 2; ++k) {
         acc = fmaf(__uint_as_float(aw[k] << 16), __uint_as_float(cw[k] << 16), acc);
         acc = fmaf(__uint_as_float(aw[k] & 0xffff0000u), __uint_as_float(cw[k] & 0xffff0000u), acc);
       }
@@ -721,6 +736,7 @@ cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
 cudaError_t launch_bwd(const BwdLaunch& L, int d, cudaStream_t stream) {
   const bool vl = L.main.cu_q != nullptr;
   if (d == 128) return vl ? launch_bwd_d<128, true>(L, stream) : launch_bwd_d<128, false>(L, stream);
+  if (d == 96) return vl ? launch_bwd_d<96, true>(L, stream) : launch_bwd_d<96, false>(L, stream);
   return vl ? launch_bwd_d<64, true>(L, stream) : launch_bwd_d<64, false>(L, stream);
 }
 

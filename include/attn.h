@@ -24,7 +24,7 @@
  *   - Head dim d is 64, 96 or 128; attn_fwd and attn_fwd_host also take 256
  *     (the "FlashAttention-2 (2023)" section's largest head dimension; its own
  *     kernel: one query tile per CTA, Q held in tensor memory); the 8-bit
- *     entry points and the backward take 64 or 128.
+ *     entry points take 64 or 128, the backward 64, 96 or 128.
  *   - Ownership: the caller owns every buffer; device pointers must stay valid
  *     until the work queued on `stream` has finished. The library allocates no
  *     device memory. `stream` is a cudaStream_t (0 = legacy default stream).
@@ -232,9 +232,9 @@ ATTN_API attn_status_t attn_q8_workspace_offsets(int B, int Hq, int Hkv, int Nq,
  *   workspace      device scratch of attn_bwd_workspace_size() bytes, 16-byte
  *                  aligned, owned by the caller; holds the fp32 dQ
  *                  accumulator, D and LSE * log2(e); needs no initial value
- * d must be 64 or 128 (96, 256: ATTN_ERR_UNSUPPORTED). The dQ accumulation adds
- * fp32 partial sums with atomics, so dQ may differ in the last bits between
- * runs; dK and dV are deterministic. Errors as attn_fwd, plus
+ * d must be 64, 96 or 128 (256: ATTN_ERR_UNSUPPORTED). The dQ accumulation
+ * adds fp32 partial sums with bulk reductions in L2 whose order is not fixed,
+ * so dQ may differ in the last bits between runs; dK and dV are deterministic. Errors as attn_fwd, plus
  * ATTN_ERR_WORKSPACE for a missing, misaligned or short workspace.
  */
 ATTN_API size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nkv, int d);

@@ -123,7 +123,7 @@ def test_bwd_entry_validation(lib):
                             ws, nbytes, None)
     assert call(dq=None) == 1 and call(dout=None) == 1 and call(Hq=3) == 1
     assert call(causal=2) == 1 and call(scale=-1.0) == 1
-    assert call(d=96) == 2 and call(d=256) == 2 and call(B=70000) == 2
+    assert call(d=80) == 2 and call(d=256) == 2 and call(B=70000) == 2
     assert call(dq=P + 4) == 3
     assert call(ws=None) == 6 and call(ws=P + 8) == 6 and call(nbytes=need - 1) == 6
 
@@ -136,6 +136,6 @@ def test_bwd_varlen_entry_validation(lib):
         return lib.attn_bwd_varlen(q, P, P, P, P, P, P, P, P, cq, P, n, mq, mk, 700, 700, 4, 2, d,
                                    causal, 0.1, ws, nbytes, None)
     assert call(cq=None) == 1 and call(n=0) == 1 and call(mq=0) == 1 and call(mk=0) == 1
-    assert call(causal=5) == 1 and call(d=96) == 2 and call(n=70000) == 2
+    assert call(causal=5) == 1 and call(d=80) == 2 and call(n=70000) == 2
     assert call(q=P + 2) == 3 and call(cq=P + 2) == 3
     assert call(ws=None) == 6 and call(nbytes=need - 1) == 6

@@ -155,6 +155,8 @@ SHAPES = [
     (1, 2, 2, 1, 257, 64, False),        # one query row
     (1, 2, 2, 1000, 1000, 128, True),
     (1, 2, 2, 129, 129, 64, True),       # one row / key past a block
+    (1, 2, 2, 300, 300, 96, True),       # d = 96: three 32-column boxes, 64-byte swizzle
+    (2, 4, 2, 200, 450, 96, False),      # d = 96, GQA 2:1, Nq < Nkv
 ]
 
 
@@ -267,6 +269,7 @@ VARLEN_BWD = [
     ([64, 200, 513], [1000, 200, 700], 4, 2, 128, True),    # prefill with a cache
     ([300, 50, 5], [100, 0, 5], 2, 2, 128, True),           # Lq > Lk, an empty key set
     ([100, 0, 37], [100, 40, 37], 2, 1, 128, True),         # an empty query sequence
+    ([1, 17, 128, 129, 300], [40, 17, 200, 129, 300], 4, 2, 96, True),  # d = 96
 ]
 
 
