@@ -34,7 +34,7 @@ from synthetic import (VARLEN_WORKLOADS, WORKLOADS, Workload, bf16_bits, make_do
 
 HEADLINE = "outlier_8k_causal"
 EXTRA_BF16 = ["tiny_256_d64", "causal_2k_d128", "outlier_8k_full", "gqa_32k_d128", "gqa_32k_d64",
-              "d256_8k_causal"]
+              "d256_8k_causal", "kvcache_128k_q128", "kvcache_128k_q128_splitkv"]
 METRIC = "attn fwd TFLOP/s (4·B·H·N²·d, causal halved), % of B200 dense BF16 peak"
 L2_BYTES = 126 * 2 ** 20
 KERNEL_SOURCES = ["exact_attention_134_b200/csrc/attn_fwd_sm100.cu",
@@ -218,6 +218,12 @@ def bench_workload(w: Workload, steps: int, warmup: int, world: int, rank: int, 
 
         def step():
             lib_mod.attn_fwd_q8(qd, kd, vd, causal=w.causal, workspace=ws, out=o, lse=lse)
+    elif w.path == "splitkv":
+        need = int(lib_mod.lib().attn_fwd_splitkv_workspace_size(wr.B, wr.Hq, wr.Nq, wr.Nkv, wr.d, 0))
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
+
+        def step():
+            lib_mod.attn_fwd_splitkv(qd, kd, vd, causal=w.causal, workspace=ws, out=o, lse=lse)
     else:
         def step():
             lib_mod.attn_fwd(qd, kd, vd, causal=w.causal, out=o, lse=lse)
@@ -430,7 +436,7 @@ def run_ours(args):
     value = aggregate_tflops(w.flops, world, ms)
     per_launch_tflops = w.flops / (statistics.mean(res["times"]) * 1e-3) / 1e12
     e2e = None
-    if not args.kernel_only and w.path != "q8":
+    if not args.kernel_only and w.path == "bf16":
         e2e_steps = max(2, args.steps // 2)
         e2e_ms, h2d, d2h = bench_e2e(w, e2e_steps, 1, world, rank, attn)
         e2e = {"value": round(world * w.flops / (e2e_ms / e2e_steps * 1e-3) / 1e12, 2),

@@ -45,6 +45,11 @@ _c_int, _c_float, _vp, _sz = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctyp
 _SIGNATURES = {
     "attn_fwd": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp]),
     "attn_fwd_varlen": (_c_int, [_vp] * 7 + [_c_int] * 8 + [_c_float, _vp]),
+    "attn_fwd_partial": (_c_int, [_vp] * 5 + [_c_int] * 7 + [_c_float, _c_int, _vp]),
+    "attn_merge_partials": (_c_int, [_vp, _vp] + [_c_int] * 5 + [_vp, _vp, _vp]),
+    "attn_fwd_splitkv_num_splits": (_c_int, [_c_int] * 5),
+    "attn_fwd_splitkv_workspace_size": (_sz, [_c_int] * 6),
+    "attn_fwd_splitkv": (_c_int, [_vp] * 5 + [_c_int] * 7 + [_c_float, _c_int, _vp, _sz, _vp]),
     "attn_fwd_host_buffer_size": (_sz, [_c_int] * 6),
     "attn_fwd_host": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp, _sz, _vp]),
     "attn_fwd_q8_workspace_size": (_sz, [_c_int] * 6),
@@ -131,6 +136,89 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None
                         B, Hq, Hkv, Nq, Nkv, d, int(bool(causal)), float(scale),
                         _stream_handle(q.device))
     _check(st, "attn_fwd")
+    return out, lse
+
+
+def _check_qkv(q, k, v):
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    return _shape_args(q, k, v)
+
+
+def attn_fwd_partial(q, k, v, causal: bool = False, scale: float | None = None, kv_tail: int = 0,
+                     out=None, lse=None):
+    """Attention of all rows of q over the keys of k, v, which are one range of
+    a longer key sequence with `kv_tail` more keys after it (the causal mask is
+    that sequence's, bottom-right aligned). Returns the range's normalised
+    partial result (o fp32 [B, Hq, Nq, d], lse fp32 [B, Hq, Nq]; -inf and
+    O = 0 for a row that sees none of its keys), for merge_partials."""
+    import torch
+    B, Hq, Hkv, Nq, Nkv, d = _check_qkv(q, k, v)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Hq, Nq, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    st = lib().attn_fwd_partial(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                lse.data_ptr(), B, Hq, Hkv, Nq, Nkv, d, int(bool(causal)),
+                                float(scale), int(kv_tail), _stream_handle(q.device))
+    _check(st, "attn_fwd_partial")
+    return out, lse
+
+
+def merge_partials(o_parts, lse_parts, out=None, lse=None):
+    """Exact merge of partial results over disjoint key ranges:
+    o_parts fp32 cuda [S, B, Hq, Nq, d], lse_parts fp32 cuda [S, B, Hq, Nq]
+    -> (o bf16 [B, Hq, Nq, d], lse fp32 [B, Hq, Nq])."""
+    import torch
+    if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32 or \
+            not o_parts.is_cuda or not lse_parts.is_cuda or \
+            not o_parts.is_contiguous() or not lse_parts.is_contiguous():
+        raise ValueError("o_parts and lse_parts must be contiguous fp32 CUDA tensors")
+    if o_parts.dim() != 5 or tuple(lse_parts.shape) != tuple(o_parts.shape[:4]):
+        raise ValueError("o_parts must be [S, B, Hq, Nq, d] and lse_parts [S, B, Hq, Nq]")
+    S, B, Hq, Nq, d = o_parts.shape
+    if out is None:
+        out = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=o_parts.device)
+    st = lib().attn_merge_partials(o_parts.data_ptr(), lse_parts.data_ptr(), S, B, Hq, Nq, d,
+                                   out.data_ptr(), lse.data_ptr(), _stream_handle(o_parts.device))
+    _check(st, "attn_merge_partials")
+    return out, lse
+
+
+def splitkv_num_splits(B, Hq, Nq, Nkv, num_splits: int = 0) -> int:
+    """Key ranges attn_fwd_splitkv uses (num_splits <= 0: its automatic choice)."""
+    return int(lib().attn_fwd_splitkv_num_splits(B, Hq, Nq, Nkv, int(num_splits)))
+
+
+def attn_fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None,
+                     num_splits: int = 0, workspace=None, out=None, lse=None):
+    """attn_fwd with the keys split into ranges computed by separate CTAs and
+    merged (for few query rows per head against many keys). Same tensors and
+    results as attn_fwd (d = 64, 96 or 128)."""
+    import torch
+    B, Hq, Hkv, Nq, Nkv, d = _check_qkv(q, k, v)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = int(lib().attn_fwd_splitkv_workspace_size(B, Hq, Nq, Nkv, d, int(num_splits)))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().attn_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                lse.data_ptr(), B, Hq, Hkv, Nq, Nkv, d, int(bool(causal)),
+                                float(scale), int(num_splits), ws_ptr, ws_len,
+                                _stream_handle(q.device))
+    _check(st, "attn_fwd_splitkv")
     return out, lse
 
 

@@ -126,9 +126,19 @@ bool make_map_u8(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
   return r == CUDA_SUCCESS;
 }
 
+// Key-range partial results (dense bf16 kernel only): o_part != null makes the
+// kernel write fp32 O rows [num_splits, B, Hq, Nq, d] and lse [num_splits, B,
+// Hq, Nq]; num_splits > 1 splits the keys into ranges of kv_chunk keys.
+struct PartialArgs {
+  float* o_part = nullptr;
+  int num_splits = 1;
+  int kv_chunk = 0;
+  int kv_tail = 0;
+};
+
 attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                       int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, const PartialArgs& part = PartialArgs()) {
   int* status = device_status_ptr();
   if (!status) return ATTN_ERR_CUDA;
   alignas(64) CUtensorMap tq, tk, tv, to;
@@ -137,7 +147,9 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
       return ATTN_ERR_CUDA;
   } else if (!make_map(&tq, q, d, Nq, (long long)B * Hq) ||
              !make_map(&tk, k, d, Nkv, (long long)B * Hkv) ||
-             !make_map(&tv, v, d, Nkv, (long long)B * Hkv) || !make_map(&to, o, d, Nq, (long long)B * Hq)) {
+             !make_map(&tv, v, d, Nkv, (long long)B * Hkv) ||
+             // a partial result is stored row by row: the output map is unused
+             !make_map(&to, part.o_part ? q : o, d, Nq, (long long)B * Hq)) {
     return ATTN_ERR_CUDA;
   }
   attn_sm100::FwdParams p;
@@ -156,6 +168,10 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.num_row_blocks = (Nq + rows - 1) / rows;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
+  p.o_part = part.o_part;
+  p.num_splits = part.num_splits;
+  p.kv_chunk = part.kv_chunk;
+  p.kv_tail = part.kv_tail;
   if (d == 256) return cuda_status(attn_sm100::launch_fwd_d256(tk, tv, q, p, stream));
   return cuda_status(attn_sm100::launch_fwd_bf16(tq, tk, tv, to, p, d, stream));
 }
@@ -445,6 +461,47 @@ attn_status_t q8_forward_with_workspace(const void* q, const void* k, const void
 
 }  // namespace attn_sm100
 
+// Split of the keys for attn_fwd_splitkv: num_splits <= 0 picks as many ranges
+// as fill one wave of CTAs (one per SM, the forward kernel's occupancy) without
+// starting a second, partly empty one; ranges hold at least two 128-key tiles.
+// The ranges are whole tiles, and only non-empty ones are launched.
+constexpr int kMaxSplits = 64;
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+struct SplitPlan {
+  int splits;
+  int chunk;
+};
+SplitPlan plan_splits(int B, int Hq, int Nq, int Nkv, int num_splits) {
+  const int tiles = (Nkv + 127) / 128;
+  long long s = num_splits;
+  if (s <= 0) {
+    const long long units = (long long)B * Hq * ((Nq + 255) / 256);
+    const long long sms = sm_count();
+    s = units >= sms ? 1 : sms / units;
+    s = std::min<long long>(s, std::max(1, tiles / 2));
+  }
+  s = std::max<long long>(1, std::min<long long>({s, (long long)tiles, (long long)kMaxSplits}));
+  const int chunk = (int)((tiles + s - 1) / s) * 128;
+  return {(Nkv + chunk - 1) / chunk, chunk};
+}
+
+struct SplitLayout {
+  size_t lse_off, total;
+};
+SplitLayout splitkv_layout(int splits, int B, int Hq, int Nq, int d) {
+  const size_t rows = (size_t)splits * B * Hq * Nq;
+  const size_t lse_off = round_up(rows * d * 4, 256);
+  return {lse_off, round_up(lse_off + rows * 4, 256)};
+}
+
 extern "C" {
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -454,6 +511,68 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   if (s != ATTN_OK) return s;
   return run_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale,
                  static_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_fwd_partial(const void* q, const void* k, const void* v, float* o_part,
+                               float* lse_part, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                               int causal, float scale, int kv_tail, void* stream) {
+  attn_status_t s = check_args(q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  if (s != ATTN_OK) return s;
+  if (kv_tail < 0 || (long long)Nkv + kv_tail > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  PartialArgs part;
+  part.o_part = o_part;
+  part.kv_tail = kv_tail;
+  return run_fwd(q, k, v, nullptr, lse_part, B, Hq, Hkv, Nq, Nkv, d, causal, scale,
+                 static_cast<cudaStream_t>(stream), part);
+}
+
+attn_status_t attn_merge_partials(const float* o_parts, const float* lse_parts, int num_parts,
+                                  int B, int Hq, int Nq, int d, void* o, float* lse,
+                                  void* stream) {
+  if (!o_parts || !lse_parts || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (num_parts <= 0 || B <= 0 || Hq <= 0 || Nq <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 96 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(o_parts) || !aligned16(lse_parts) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_ALIGNMENT;
+  return cuda_status(attn_sm100::launch_merge(o_parts, lse_parts, num_parts,
+                                              (long long)B * Hq * Nq, d, o, lse,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int attn_fwd_splitkv_num_splits(int B, int Hq, int Nq, int Nkv, int num_splits) {
+  if (B <= 0 || Hq <= 0 || Nq <= 0 || Nkv <= 0) return 0;
+  return plan_splits(B, Hq, Nq, Nkv, num_splits).splits;
+}
+
+size_t attn_fwd_splitkv_workspace_size(int B, int Hq, int Nq, int Nkv, int d, int num_splits) {
+  if (B <= 0 || Hq <= 0 || Nq <= 0 || Nkv <= 0 || d <= 0) return 0;
+  const SplitPlan plan = plan_splits(B, Hq, Nq, Nkv, num_splits);
+  return plan.splits == 1 ? 0 : splitkv_layout(plan.splits, B, Hq, Nq, d).total;
+}
+
+attn_status_t attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int Hq, int Hkv, int Nq, int Nkv, int d, int causal,
+                               float scale, int num_splits, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  if (s != ATTN_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const SplitPlan plan = plan_splits(B, Hq, Nq, Nkv, num_splits);
+  if (plan.splits == 1) return run_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, st);
+  if ((long long)B * plan.splits > 65535) return ATTN_ERR_UNSUPPORTED;
+  const SplitLayout lay = splitkv_layout(plan.splits, B, Hq, Nq, d);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < lay.total) return ATTN_ERR_WORKSPACE;
+  uint8_t* const ws = static_cast<uint8_t*>(workspace);
+  float* const o_parts = reinterpret_cast<float*>(ws);
+  float* const lse_parts = reinterpret_cast<float*>(ws + lay.lse_off);
+  PartialArgs part;
+  part.o_part = o_parts;
+  part.num_splits = plan.splits;
+  part.kv_chunk = plan.chunk;
+  s = run_fwd(q, k, v, nullptr, lse_parts, B, Hq, Hkv, Nq, Nkv, d, causal, scale, st, part);
+  if (s != ATTN_OK) return s;
+  return cuda_status(attn_sm100::launch_merge(o_parts, lse_parts, plan.splits,
+                                              (long long)B * Hq * Nq, d, o, lse, st));
 }
 
 attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -154,19 +154,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     Lq = min(max(p.cu_q[sq + 1], q_start), p.Nq) - q_start;
     k_start = min(max(p.cu_k[sq], 0), p.Nkv);
     Lk = min(max(p.cu_k[sq + 1], k_start), p.Nkv) - k_start;
+  } else if (p.num_splits > 1) {
+    // key range (blockIdx.z % num_splits) of a partial-result launch
+    k_start = ((int)blockIdx.z % p.num_splits) * p.kv_chunk;  // < Nkv: only non-empty ranges are launched
+    Lk = min(p.Nkv - k_start, p.kv_chunk);
   }
   const int nrb = (Lq + 2 * kBM - 1) / (2 * kBM);
   if ((int)blockIdx.x >= nrb) return;  // this sequence has fewer rows (the whole CTA leaves)
   const int row_block = p.causal ? (nrb - 1 - (int)blockIdx.x) : (int)blockIdx.x;
   const int hq = blockIdx.y;
-  const int b = VL ? 0 : (int)blockIdx.z;
+  const int b = VL ? 0 : (int)blockIdx.z / p.num_splits;
   const int hk = hq / (p.Hq / p.Hkv);
   const int q0 = row_block * 2 * kBM;  // first query row of the unit, within its sequence
   const int bh_q = b * p.Hq + hq;
   const int bh_kv = b * p.Hkv + hk;
-  // causal mask aligned to the bottom right: key j is visible to query i iff
-  // j <= i + (Lk - Lq)
-  const int diag = p.causal ? Lk - Lq : 0;
+  // causal mask aligned to the bottom right of the full key sequence: key j
+  // (of this unit's range) is visible to query i iff j <= i + (Lk + tail - Lq),
+  // tail = the keys after the range (0 unless the keys are split)
+  const int tail = VL ? 0 : p.kv_tail + (p.Nkv - k_start - Lk);
+  const int diag = p.causal ? Lk + tail - Lq : 0;
   // K/V tiles a query tile needs (at least one, so every pipeline runs; a row
   // that sees no key ends with l = 0): all of them, or (causal) up to the key
   // its last row sees. Query tile 0 of a causal CTA thus skips the last tile.
@@ -180,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // TMA coordinates (rows, outer) of a query tile / a K/V tile
   const int q_c1 = VL ? hq : 0, kv_c1 = VL ? hk : 0;
   auto q_row = [&](int t) { return VL ? q_start + q0 + t * kBM : q0 + t * kBM; };
-  auto kv_row = [&](int j) { return VL ? k_start + j * kBN : j * kBN; };
+  auto kv_row = [&](int j) { return k_start + j * kBN; };
   const uint64_t budget = p.timeout_ns;
 
   // ---- setup: barriers (thread 0), TMEM (MMA warp)
@@ -425,7 +431,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (ok) ok = warp_all(bounded_wait(bar(BarLayout::kOFinal), 0, abort_flag, budget));
-    if (ok && (VL || C::kRowStores)) {
+    if (ok && !VL && p.o_part != nullptr) {
+      // ---- epilogue of a partial result: O = O_acc / l in fp32, row by row;
+      // a row that saw no key of the range gets O = 0, LSE = -inf
+      tc_fence_after();
+      const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+      const bool valid = row < Lq;
+      const int split = p.num_splits > 1 ? (int)blockIdx.z % p.num_splits : 0;
+      const size_t prow = ((size_t)split * p.B * p.Hq + bh_q) * p.Nq + (valid ? row : 0);
+      float4* const orow = reinterpret_cast<float4*>(p.o_part + prow * D);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * c, o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            orow[c * 8 + q] = make_float4(__uint_as_float(o[4 * q]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
+                                          __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
+        }
+      }
+      if (valid) p.lse[prow] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+    } else if (ok && (VL || C::kRowStores)) {
       // ---- epilogue (packed sequences, d = 96): O = O_acc / l -> bf16 stored row by row
       tc_fence_after();
       const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
@@ -514,7 +542,7 @@ static cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, co
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_bf16_kernel<D, VL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<D>());
   if (e != cudaSuccess) return e;
-  dim3 grid(p.num_row_blocks, p.Hq, p.B);  // varlen: B = number of sequences
+  dim3 grid(p.num_row_blocks, p.Hq, p.B * p.num_splits);  // varlen: B = number of sequences
   attn_fwd_bf16_kernel<D, VL><<<grid, kThreads, smem_bytes<D>(), stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }

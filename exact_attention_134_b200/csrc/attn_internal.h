@@ -22,6 +22,12 @@ struct FwdParams {
   int num_row_blocks;             // ceil(Nq / rows per work unit); packed: of the longest sequence
   float scale_log2;               // scale * log2(e)
   unsigned long long timeout_ns;  // budget of every pipeline wait
+  // Partial results over key ranges (dense tensors only; see attn_fwd_partial):
+  float* o_part = nullptr;        // fp32 O rows [num_splits, B, Hq, Nq, d] instead of bf16 o;
+                                  // lse is then [num_splits, B, Hq, Nq]
+  int num_splits = 1;             // key ranges per (b, h): grid z = B * num_splits
+  int kv_chunk = 0;               // keys per range (a multiple of 128) when num_splits > 1
+  int kv_tail = 0;                // keys after this K/V tensor in the full sequence (causal)
 };
 
 // Kernel parameters of the 8-bit main kernel.
@@ -121,6 +127,12 @@ attn_status_t q8_forward_with_workspace(const void* q, const void* k, const void
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t stream);
 int fwd_rows_per_cta();
+
+// O = sum_s exp(LSE_s - LSE) O_s, LSE = ln sum_s exp(LSE_s) over num_parts
+// partial results [num_parts, rows, d] fp32 / [num_parts, rows] fp32;
+// writes bf16 O [rows, d] and fp32 LSE [rows].
+cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int num_parts,
+                         long long rows, int d, void* o, float* lse, cudaStream_t stream);
 
 // Head dim 256 (dense tensors only): K/V tensor maps with 64-row boxes; Q is
 // read directly from global memory.

@@ -101,6 +101,69 @@ ATTN_API attn_status_t attn_fwd_varlen(const void* q, const void* k, const void*
                                        void* stream);
 
 /*
+ * Key-range partial results and their merge ("FlashAttention (TR)", section
+ * "Çevrimiçi Softmax Hesaplama": the running maximum / running sum update,
+ * applied to whole key ranges). For disjoint key ranges s with normalised
+ * partial outputs O_s and LSE_s = ln sum_{j in s} exp(scale q.k_j):
+ *     LSE = ln sum_s exp(LSE_s),   O = sum_s exp(LSE_s - LSE) O_s,
+ * which is exactly attn_fwd over the union of the ranges.
+ *
+ * attn_fwd_partial — attn_fwd of all Nq query rows over the Nkv keys of k, v
+ * when those keys are one range [lo, lo + Nkv) of a longer sequence that has
+ * kv_tail >= 0 more keys after them (a key-sharded multi-GPU forward: each
+ * rank holds one range). The causal mask is the full sequence's, aligned to
+ * its bottom right: key lo + j is visible to query i iff
+ * lo + j <= i + (lo + Nkv + kv_tail - Nq), i.e. j <= i + Nkv + kv_tail - Nq
+ * (kv_tail = 0: exactly attn_fwd's mask).
+ *   q, k, v   as attn_fwd (d = 64, 96 or 128)
+ *   o_part    device, fp32 [B, Hq, Nq, d]   (written; normalised over the range)
+ *   lse_part  device, fp32 [B, Hq, Nq]      (written; -inf, with O = 0, for a
+ *                                            row that sees no key of the range)
+ * Allocates nothing; one kernel launch on `stream`.
+ */
+ATTN_API attn_status_t attn_fwd_partial(const void* q, const void* k, const void* v,
+                                        float* o_part, float* lse_part, int B, int Hq, int Hkv,
+                                        int Nq, int Nkv, int d, int causal, float scale,
+                                        int kv_tail, void* stream);
+
+/*
+ * attn_merge_partials — the merge above over num_parts results stacked along
+ * a leading axis (e.g. an all-gather of the ranks' attn_fwd_partial outputs,
+ * in any order).
+ *   o_parts    device, fp32 [num_parts, B, Hq, Nq, d]
+ *   lse_parts  device, fp32 [num_parts, B, Hq, Nq]
+ *   o          device, bf16 [B, Hq, Nq, d]   (written; RNE from fp32)
+ *   lse        device, fp32 [B, Hq, Nq]      (written)
+ * d = 64, 96, 128 or 256. One kernel launch; allocates nothing.
+ */
+ATTN_API attn_status_t attn_merge_partials(const float* o_parts, const float* lse_parts,
+                                           int num_parts, int B, int Hq, int Nq, int d, void* o,
+                                           float* lse, void* stream);
+
+/*
+ * attn_fwd_splitkv — attn_fwd with the keys split into ranges that run as
+ * separate CTAs of one launch, then merged: for shapes with few query rows
+ * per head and many keys (prefill against a long cache), where attn_fwd's
+ * B * Hq * ceil(Nq / 256) CTAs would leave SMs idle. Same arguments and
+ * results as attn_fwd (d = 64, 96 or 128), plus
+ *   num_splits  key ranges per (b, h); <= 0 picks floor(SMs / CTAs of
+ *               attn_fwd) ranges, one full wave (ranges of whole 128-key
+ *               tiles, at least two tiles each, at most 64 ranges);
+ *               attn_fwd_splitkv_num_splits() returns
+ *               the count used (1 = plain attn_fwd, no workspace needed)
+ *   workspace   device scratch of attn_fwd_splitkv_workspace_size() bytes,
+ *               16-byte aligned, owned by the caller: the fp32 partials
+ * Two launches (partials, merge). ATTN_ERR_UNSUPPORTED if B * ranges > 65535.
+ */
+ATTN_API int attn_fwd_splitkv_num_splits(int B, int Hq, int Nq, int Nkv, int num_splits);
+ATTN_API size_t attn_fwd_splitkv_workspace_size(int B, int Hq, int Nq, int Nkv, int d,
+                                                int num_splits);
+ATTN_API attn_status_t attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
+                                        float* lse, int B, int Hq, int Hkv, int Nq, int Nkv,
+                                        int d, int causal, float scale, int num_splits,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * attn_fwd_host — the same operation on HOST buffers, for callers whose data
  * lives in host memory. Copies q, k, v into `dev_buf` (a device buffer of at
  * least attn_fwd_host_buffer_size() bytes, 16-byte aligned, owned by the

@@ -39,7 +39,7 @@ class Workload:
     causal: bool
     seed: int
     dist: str = "normal"          # "normal" | "outlier_k"
-    path: str = "bf16"            # "bf16" | "q8" (8-bit mainloop)
+    path: str = "bf16"            # "bf16" | "q8" (8-bit mainloop) | "splitkv" (split keys)
     oracle_rows: int = 0          # 0 = every query row; else rows sampled per (b, hq)
 
     @property
@@ -80,6 +80,12 @@ WORKLOADS = {
     # head dim 256 (the largest the FlashAttention-2 section names), 8k causal
     "d256_8k_causal": Workload("d256_8k_causal", 1, 16, 16, 8192, 8192, 256, True, 1008,
                                oracle_rows=64),
+    # 128 new query rows against a 128k-key cache (GQA 32/8): too few CTAs for
+    # the row-parallel forward; the same inputs through the split-key forward
+    "kvcache_128k_q128": Workload("kvcache_128k_q128", 1, 32, 8, 128, 131072, 128, False, 1010,
+                                  oracle_rows=8),
+    "kvcache_128k_q128_splitkv": Workload("kvcache_128k_q128_splitkv", 1, 32, 8, 128, 131072, 128,
+                                          False, 1010, path="splitkv", oracle_rows=8),
 }
 
 

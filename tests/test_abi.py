@@ -139,3 +139,39 @@ def test_bwd_varlen_entry_validation(lib):
     assert call(causal=5) == 1 and call(d=80) == 2 and call(n=70000) == 2
     assert call(q=P + 2) == 3 and call(cq=P + 2) == 3
     assert call(ws=None) == 6 and call(nbytes=need - 1) == 6
+
+
+def test_partial_and_merge_entry_validation(lib):
+    def partial(q=P, o=P, lse=P, d=128, tail=0, Nkv=500):
+        return lib.attn_fwd_partial(q, P, P, o, lse, 1, 4, 2, 300, Nkv, d, 1, 0.1, tail, None)
+    assert partial(o=None) == 1 and partial(lse=None) == 1 and partial(tail=-1) == 1
+    assert partial(Nkv=0) == 1 and partial(Nkv=2 ** 31 - 10, tail=20) == 1
+    assert partial(d=256) == 2 and partial(d=80) == 2
+    assert partial(q=P + 2) == 3 and partial(o=P + 4) == 3
+
+    def merge(op=P, lp=P, n=3, d=128, o=P, lse=P, B=2):
+        return lib.attn_merge_partials(op, lp, n, B, 4, 300, d, o, lse, None)
+    assert merge(op=None) == 1 and merge(o=None) == 1 and merge(n=0) == 1 and merge(B=0) == 1
+    assert merge(d=80) == 2 and merge(d=512) == 2
+    assert merge(lp=P + 4) == 3 and merge(o=P + 8) == 3
+
+
+def test_splitkv_plan_and_validation(lib):
+    # the automatic choice fills one wave of CTAs (at most 148 here: without a
+    # GPU the library assumes 148 SMs) with ranges of at least two key tiles
+    assert attn.splitkv_num_splits(1, 32, 128, 131072) == 4      # 32 CTAs -> 4 ranges
+    assert attn.splitkv_num_splits(2, 32, 8192, 8192) == 1       # already > 148 CTAs
+    assert attn.splitkv_num_splits(1, 1, 16, 1 << 20) == 64      # capped at 64 ranges
+    assert attn.splitkv_num_splits(1, 2, 10, 300) == 1           # 3 tiles: ranges of >= 2
+    assert attn.splitkv_num_splits(1, 2, 10, 1000, 5) == 4       # 8 tiles in ranges of 2
+    assert attn.splitkv_num_splits(1, 2, 10, 1000, 100) == 8     # at most one range per tile
+    assert attn.splitkv_num_splits(0, 2, 10, 1000) == 0
+    need = lib.attn_fwd_splitkv_workspace_size(1, 32, 128, 131072, 128, 0)
+    assert need >= 4 * 32 * 128 * (128 + 1) * 4 and need % 256 == 0
+    assert lib.attn_fwd_splitkv_workspace_size(2, 32, 8192, 8192, 128, 0) == 0  # one range
+
+    def call(ws=P, nbytes=need, d=128, B=1, S=0):
+        return lib.attn_fwd_splitkv(P, P, P, P, P, B, 32, 8, 128, 131072, d, 0, 0.1, S, ws,
+                                    nbytes, None)
+    assert call(ws=None) == 6 and call(ws=P + 8) == 6 and call(nbytes=need - 1) == 6
+    assert call(d=256) == 2 and call(B=20000, S=64) == 2

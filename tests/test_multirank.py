@@ -89,3 +89,80 @@ def test_reference_arm_rank0_json(capsys, monkeypatch):
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["config"]["workload"] == "tiny_256_d64"
+
+
+# ---------------------------------------------------------------- key-sharded forward
+
+def test_shard_bounds_cover_the_keys_in_rank_order():
+    from exact_attention_134_b200.kv_shard import shard_bounds
+    for n in (1, 7, 128, 1000, 8193):
+        for world in (1, 2, 3, 8):
+            b = [shard_bounds(n, world, r) for r in range(world)]
+            assert b[0][0] == 0 and b[-1][1] == n
+            assert all(b[r][1] == b[r + 1][0] for r in range(world - 1))
+            sizes = [hi - lo for lo, hi in b]
+            assert max(sizes) - min(sizes) <= 1 and sizes == sorted(sizes, reverse=True)
+
+
+def _oracle_partial(q, k, v, causal, scale, kv_tail):
+    """The partial a rank computes, from the oracle: its keys padded with
+    kv_tail dummy keys after them (they only move the causal alignment)."""
+    import numpy as np
+    from oracle import attention_partial_fp64
+    from synthetic import bf16_bits
+    pad = torch.zeros((k.shape[0], k.shape[1], kv_tail, k.shape[3]), dtype=k.dtype)
+    kb, vb = bf16_bits(torch.cat([k, pad], 2)), bf16_bits(torch.cat([v, pad], 2))
+    o, lse = attention_partial_fp64(bf16_bits(q), kb, vb, 0, k.shape[2], causal, scale)
+    return torch.from_numpy(np.ascontiguousarray(o)), torch.from_numpy(np.ascontiguousarray(lse))
+
+
+def _oracle_merge(o_all, lse_all):
+    from oracle import merge_partials_fp64
+    o, lse = merge_partials_fp64(o_all.numpy(), lse_all.numpy())
+    return torch.from_numpy(o), torch.from_numpy(lse)
+
+
+def _kv_worker(rank, world, port, causal, out):
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    import torch.distributed as dist
+    from exact_attention_134_b200.kv_shard import attention_kv_sharded, shard_bounds
+    from synthetic import make_qkv
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    n_keys = 301
+    q, k, v = make_qkv(1, 4, 2, 40, n_keys, 16, seed=31)   # every rank draws the same tensors
+    lo, hi = shard_bounds(n_keys, world, rank)
+    o, lse = attention_kv_sharded(q, k[:, :, lo:hi].contiguous(), v[:, :, lo:hi].contiguous(),
+                                  n_keys, causal=causal, scale=0.25,
+                                  partial_fn=_oracle_partial, merge_fn=_oracle_merge)
+    out[rank] = (o.numpy(), lse.numpy())
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_kv_sharded_three_ranks_gloo(causal):
+    """Three gloo ranks, each holding a third of the keys: the gathered and
+    merged partials equal the full attention on every rank (the exchange's
+    order, the ranges and the causal tails are what is checked)."""
+    if torch.cuda.is_available():
+        pytest.skip("CPU/gloo test")
+    import numpy as np
+    from oracle import attention_fp64
+    from synthetic import bf16_bits, make_qkv
+    world = 3
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        procs = [ctx.Process(target=_kv_worker, args=(r, world, port, causal, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(120)
+            assert p.exitcode == 0
+        res = dict(out)
+    q, k, v = make_qkv(1, 4, 2, 40, 301, 16, seed=31)
+    O, L = attention_fp64(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, 0.25)
+    for r in range(world):
+        o, lse = res[r]
+        assert np.abs(o - O).max() < 1e-12 and np.abs(lse - L).max() < 1e-12
