@@ -219,7 +219,8 @@ def bench_workload(w: Workload, steps: int, warmup: int, world: int, rank: int, 
         def step():
             lib_mod.attn_fwd_q8(qd, kd, vd, causal=w.causal, workspace=ws, out=o, lse=lse)
     elif w.path == "splitkv":
-        need = int(lib_mod.lib().attn_fwd_splitkv_workspace_size(wr.B, wr.Hq, wr.Nq, wr.Nkv, wr.d, 0))
+        need = int(lib_mod.lib().attn_fwd_splitkv_workspace_size(wr.B, wr.Hq, wr.Hkv, wr.Nq, wr.Nkv,
+                                                                   wr.d, 0))
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
 
         def step():

@@ -47,8 +47,8 @@ _SIGNATURES = {
     "attn_fwd_varlen": (_c_int, [_vp] * 7 + [_c_int] * 8 + [_c_float, _vp]),
     "attn_fwd_partial": (_c_int, [_vp] * 5 + [_c_int] * 7 + [_c_float, _c_int, _vp]),
     "attn_merge_partials": (_c_int, [_vp, _vp] + [_c_int] * 5 + [_vp, _vp, _vp]),
-    "attn_fwd_splitkv_num_splits": (_c_int, [_c_int] * 5),
-    "attn_fwd_splitkv_workspace_size": (_sz, [_c_int] * 6),
+    "attn_fwd_splitkv_num_splits": (_c_int, [_c_int] * 7),
+    "attn_fwd_splitkv_workspace_size": (_sz, [_c_int] * 7),
     "attn_fwd_splitkv": (_c_int, [_vp] * 5 + [_c_int] * 7 + [_c_float, _c_int, _vp, _sz, _vp]),
     "attn_fwd_host_buffer_size": (_sz, [_c_int] * 6),
     "attn_fwd_host": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp, _sz, _vp]),
@@ -191,9 +191,9 @@ def merge_partials(o_parts, lse_parts, out=None, lse=None):
     return out, lse
 
 
-def splitkv_num_splits(B, Hq, Nq, Nkv, num_splits: int = 0) -> int:
+def splitkv_num_splits(B, Hq, Hkv, Nq, Nkv, d, num_splits: int = 0) -> int:
     """Key ranges attn_fwd_splitkv uses (num_splits <= 0: its automatic choice)."""
-    return int(lib().attn_fwd_splitkv_num_splits(B, Hq, Nq, Nkv, int(num_splits)))
+    return int(lib().attn_fwd_splitkv_num_splits(B, Hq, Hkv, Nq, Nkv, d, int(num_splits)))
 
 
 def attn_fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None,
@@ -205,7 +205,7 @@ def attn_fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None,
     B, Hq, Hkv, Nq, Nkv, d = _check_qkv(q, k, v)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    need = int(lib().attn_fwd_splitkv_workspace_size(B, Hq, Nq, Nkv, d, int(num_splits)))
+    need = int(lib().attn_fwd_splitkv_workspace_size(B, Hq, Hkv, Nq, Nkv, d, int(num_splits)))
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     if out is None:

@@ -136,6 +136,18 @@ struct PartialArgs {
   int kv_tail = 0;
 };
 
+// A CTA of the bf16 forward holds two 128-row query tiles: 256 rows of one
+// query head, or — for Nq <= 128 with an even number of query heads per kv
+// head — the same rows of two query heads that share their K/V tiles.
+bool pairs_heads(int Hq, int Hkv, int Nq, int d) {
+  return d != 256 && Nq <= attn_sm100::fwd_rows_per_cta_paired() && (Hq / Hkv) % 2 == 0;
+}
+long long fwd_ctas(int B, int Hq, int Hkv, int Nq, int d) {
+  if (pairs_heads(Hq, Hkv, Nq, d)) return (long long)B * (Hq / 2);
+  const int rows = attn_sm100::fwd_rows_per_cta();
+  return (long long)B * Hq * ((Nq + rows - 1) / rows);
+}
+
 attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                       int Hq, int Hkv, int Nq, int Nkv, int d, int causal, float scale,
                       cudaStream_t stream, const PartialArgs& part = PartialArgs()) {
@@ -164,7 +176,9 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.causal = causal;
-  const int rows = attn_sm100::fwd_rows_per_cta();
+  // short query blocks: pair the query heads of a kv head in one CTA
+  p.pair_heads = pairs_heads(Hq, Hkv, Nq, d) ? 1 : 0;
+  const int rows = p.pair_heads ? attn_sm100::fwd_rows_per_cta_paired() : attn_sm100::fwd_rows_per_cta();
   p.num_row_blocks = (Nq + rows - 1) / rows;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
@@ -479,11 +493,11 @@ struct SplitPlan {
   int splits;
   int chunk;
 };
-SplitPlan plan_splits(int B, int Hq, int Nq, int Nkv, int num_splits) {
+SplitPlan plan_splits(int B, int Hq, int Hkv, int Nq, int Nkv, int d, int num_splits) {
   const int tiles = (Nkv + 127) / 128;
   long long s = num_splits;
   if (s <= 0) {
-    const long long units = (long long)B * Hq * ((Nq + 255) / 256);
+    const long long units = fwd_ctas(B, Hq, Hkv, Nq, d);
     const long long sms = sm_count();
     s = units >= sms ? 1 : sms / units;
     s = std::min<long long>(s, std::max(1, tiles / 2));
@@ -539,14 +553,15 @@ attn_status_t attn_merge_partials(const float* o_parts, const float* lse_parts, 
                                               static_cast<cudaStream_t>(stream)));
 }
 
-int attn_fwd_splitkv_num_splits(int B, int Hq, int Nq, int Nkv, int num_splits) {
-  if (B <= 0 || Hq <= 0 || Nq <= 0 || Nkv <= 0) return 0;
-  return plan_splits(B, Hq, Nq, Nkv, num_splits).splits;
+int attn_fwd_splitkv_num_splits(int B, int Hq, int Hkv, int Nq, int Nkv, int d, int num_splits) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Nq <= 0 || Nkv <= 0 || d <= 0) return 0;
+  return plan_splits(B, Hq, Hkv, Nq, Nkv, d, num_splits).splits;
 }
 
-size_t attn_fwd_splitkv_workspace_size(int B, int Hq, int Nq, int Nkv, int d, int num_splits) {
-  if (B <= 0 || Hq <= 0 || Nq <= 0 || Nkv <= 0 || d <= 0) return 0;
-  const SplitPlan plan = plan_splits(B, Hq, Nq, Nkv, num_splits);
+size_t attn_fwd_splitkv_workspace_size(int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                                       int num_splits) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Nq <= 0 || Nkv <= 0 || d <= 0) return 0;
+  const SplitPlan plan = plan_splits(B, Hq, Hkv, Nq, Nkv, d, num_splits);
   return plan.splits == 1 ? 0 : splitkv_layout(plan.splits, B, Hq, Nq, d).total;
 }
 
@@ -557,7 +572,7 @@ attn_status_t attn_fwd_splitkv(const void* q, const void* k, const void* v, void
   attn_status_t s = check_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
   if (s != ATTN_OK) return s;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const SplitPlan plan = plan_splits(B, Hq, Nq, Nkv, num_splits);
+  const SplitPlan plan = plan_splits(B, Hq, Hkv, Nq, Nkv, d, num_splits);
   if (plan.splits == 1) return run_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal, scale, st);
   if ((long long)B * plan.splits > 65535) return ATTN_ERR_UNSUPPORTED;
   const SplitLayout lay = splitkv_layout(plan.splits, B, Hq, Nq, d);

@@ -123,7 +123,16 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
 // VL = true : packed variable-length sequences [total, H, d]; grid z = sequence,
 //             its query/key rows come from cu_seqlens; O and LSE are stored
 //             row by row (a TMA box could cross into the next sequence).
-template <int D, bool VL>
+// PART = true (dense only): a partial result over key ranges — grid z = batch
+//             entry x range, fp32 O rows and LSE per range, the causal mask
+//             aligned to the end of the full key sequence (p.kv_tail keys
+//             after the tensor). A separate instantiation, so the plain
+//             forward carries none of it.
+// PAIR = true (dense, Nq <= 128, an even number of query heads per kv head):
+//             the two query tiles are the same rows of two query heads that
+//             share a kv head (2 * blockIdx.y and 2 * blockIdx.y + 1), so a
+//             short query block does not leave the second tile empty.
+template <int D, bool VL, bool PART, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -154,24 +163,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     Lq = min(max(p.cu_q[sq + 1], q_start), p.Nq) - q_start;
     k_start = min(max(p.cu_k[sq], 0), p.Nkv);
     Lk = min(max(p.cu_k[sq + 1], k_start), p.Nkv) - k_start;
-  } else if (p.num_splits > 1) {
+  } else if (PART && p.num_splits > 1) {
     // key range (blockIdx.z % num_splits) of a partial-result launch
     k_start = ((int)blockIdx.z % p.num_splits) * p.kv_chunk;  // < Nkv: only non-empty ranges are launched
     Lk = min(p.Nkv - k_start, p.kv_chunk);
   }
-  const int nrb = (Lq + 2 * kBM - 1) / (2 * kBM);
+  constexpr int kUnitRows = PAIR ? kBM : 2 * kBM;  // query rows of a work unit
+  constexpr int kTileRowStep = PAIR ? 0 : kBM;    // first row of tile 1 - of tile 0
+  const int nrb = (Lq + kUnitRows - 1) / kUnitRows;
   if ((int)blockIdx.x >= nrb) return;  // this sequence has fewer rows (the whole CTA leaves)
   const int row_block = p.causal ? (nrb - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-  const int hq = blockIdx.y;
-  const int b = VL ? 0 : (int)blockIdx.z / p.num_splits;
+  const int hq = PAIR ? 2 * (int)blockIdx.y : (int)blockIdx.y;  // query head of tile 0
+  const int b = VL ? 0 : (PART ? (int)blockIdx.z / p.num_splits : (int)blockIdx.z);
   const int hk = hq / (p.Hq / p.Hkv);
-  const int q0 = row_block * 2 * kBM;  // first query row of the unit, within its sequence
-  const int bh_q = b * p.Hq + hq;
+  const int q0 = row_block * kUnitRows;  // first query row of the unit, within its sequence
+  const int bh_q = b * p.Hq + hq;        // (tile 1: bh_q + 1 when PAIR)
   const int bh_kv = b * p.Hkv + hk;
   // causal mask aligned to the bottom right of the full key sequence: key j
   // (of this unit's range) is visible to query i iff j <= i + (Lk + tail - Lq),
   // tail = the keys after the range (0 unless the keys are split)
-  const int tail = VL ? 0 : p.kv_tail + (p.Nkv - k_start - Lk);
+  const int tail = PART ? p.kv_tail + (p.Nkv - k_start - Lk) : 0;
   const int diag = p.causal ? Lk + tail - Lq : 0;
   // K/V tiles a query tile needs (at least one, so every pipeline runs; a row
   // that sees no key ends with l = 0): all of them, or (causal) up to the key
@@ -181,11 +192,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int last_key = min(last_row + diag, Lk - 1);
     return last_key < 0 ? 1 : last_key / kBN + 1;
   };
-  const int n_tiles = tiles_for(min(q0 + 2 * kBM - 1, Lq - 1));
-  const int n_tiles0 = tiles_for(min(q0 + kBM - 1, Lq - 1));
+  const int n_tiles = tiles_for(min(q0 + kUnitRows - 1, Lq - 1));
+  const int n_tiles0 = PAIR ? n_tiles : tiles_for(min(q0 + kBM - 1, Lq - 1));
   // TMA coordinates (rows, outer) of a query tile / a K/V tile
   const int q_c1 = VL ? hq : 0, kv_c1 = VL ? hk : 0;
-  auto q_row = [&](int t) { return VL ? q_start + q0 + t * kBM : q0 + t * kBM; };
+  auto q_row = [&](int t) { return VL ? q_start + q0 + t * kBM : q0 + t * kTileRowStep; };
   auto kv_row = [&](int j) { return k_start + j * kBN; };
   const uint64_t budget = p.timeout_ns;
 
@@ -230,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < 2; ++t)
         for (int bx = 0; bx < C::kBoxes; ++bx)
           tma_load_3d(sQ + t * C::kTileBytes + bx * C::kBoxBytes, &tm_q, bar(BarLayout::kQFull),
-                      bx * C::kBoxCols, VL ? q_c1 : q_row(t), VL ? q_row(t) : bh_q);
+                      bx * C::kBoxCols, VL ? q_c1 : q_row(t), VL ? q_row(t) : bh_q + (PAIR ? t : 0));
     }
     for (int j = 0; j < n_tiles && ok; ++j) {
       for (int which = 0; which < 2; ++which) {  // 0 = K_j, 1 = V_j
@@ -356,7 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(wq << 5) << 16;
     const uint32_t tS = tmem + (t ? C::kColS1 : C::kColS0) + lane_off;
     const uint32_t tO = tmem + (t ? C::kColO1 : C::kColO0) + lane_off;
-    const int row = q0 + t * kBM + r;
+    const int row = q0 + t * kTileRowStep + r;
+    const int bh_qt = bh_q + (PAIR ? t : 0);  // this tile's (batch, query head)
     const float sl2 = p.scale_log2;
 
     float m_run = -INFINITY;  // reference maximum of scale*log2(e)*S over the row, so far
@@ -431,14 +443,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (ok) ok = warp_all(bounded_wait(bar(BarLayout::kOFinal), 0, abort_flag, budget));
-    if (ok && !VL && p.o_part != nullptr) {
+    if (PART && ok) {
       // ---- epilogue of a partial result: O = O_acc / l in fp32, row by row;
       // a row that saw no key of the range gets O = 0, LSE = -inf
       tc_fence_after();
       const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
       const bool valid = row < Lq;
       const int split = p.num_splits > 1 ? (int)blockIdx.z % p.num_splits : 0;
-      const size_t prow = ((size_t)split * p.B * p.Hq + bh_q) * p.Nq + (valid ? row : 0);
+      const size_t prow = ((size_t)split * p.B * p.Hq + bh_qt) * p.Nq + (valid ? row : 0);
       float4* const orow = reinterpret_cast<float4*>(p.o_part + prow * D);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
@@ -459,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
       const bool valid = row < Lq;  // q_start + row < total holds by the clamping above
       const size_t orow_idx = VL ? (size_t)(q_start + (valid ? row : 0)) * p.Hq + hq
-                                 : (size_t)bh_q * p.Nq + (valid ? row : 0);
+                                 : (size_t)bh_qt * p.Nq + (valid ? row : 0);
       uint4* const orow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow_idx * D);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
@@ -479,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (valid)  // LSE: packed sequences [Hq, total_q], dense [B, Hq, Nq]
-        p.lse[VL ? (size_t)hq * p.Nq + q_start + row : (size_t)bh_q * p.Nq + row] =
+        p.lse[VL ? (size_t)hq * p.Nq + q_start + row : (size_t)bh_qt * p.Nq + row] =
             (m_run + log2f(l_run)) * 0.69314718055994530942f;
     } else if (ok) {
       // ---- epilogue: O = O_acc / l -> bf16 into the (now free) Q_t buffer, then TMA store
@@ -506,12 +518,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(BarLayout::kEpi + t));
-      if (row < Lq) p.lse[(size_t)bh_q * p.Nq + row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+      if (row < Lq) p.lse[(size_t)bh_qt * p.Nq + row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
       if (r == 0) {
         volatile int no_abort = 0;
         if (bounded_wait(bar(BarLayout::kEpi + t), 0, &no_abort, budget)) {
           for (int bx = 0; bx < C::kBoxes; ++bx)
-            tma_store_3d(&tm_o, sQ + t * C::kTileBytes + bx * C::kBoxBytes, bx * 64, q0 + t * kBM, bh_q);
+            tma_store_3d(&tm_o, sQ + t * C::kTileBytes + bx * C::kBoxBytes, bx * 64, q0 + t * kTileRowStep,
+                         bh_qt);
           tma_store_commit();
           tma_store_wait_all();
         } else {
@@ -536,20 +549,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 static int smem_bytes() { return FwdCfg<D>::kSmemBytes; }
 
-template <int D, bool VL>
+template <int D, bool VL, bool PART = false, bool PAIR = false>
 static cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& to, const FwdParams& p, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_bf16_kernel<D, VL>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_bf16_kernel<D, VL, PART, PAIR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<D>());
   if (e != cudaSuccess) return e;
-  dim3 grid(p.num_row_blocks, p.Hq, p.B * p.num_splits);  // varlen: B = number of sequences
-  attn_fwd_bf16_kernel<D, VL><<<grid, kThreads, smem_bytes<D>(), stream>>>(tq, tk, tv, to, p);
+  // varlen: B = number of sequences; head pairs: Hq / 2 units of 128 rows
+  dim3 grid(p.num_row_blocks, PAIR ? p.Hq / 2 : p.Hq, p.B * p.num_splits);
+  attn_fwd_bf16_kernel<D, VL, PART, PAIR><<<grid, kThreads, smem_bytes<D>(), stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t stream) {
   const bool vl = p.cu_q != nullptr;
+  if (!vl && p.pair_heads) {  // dense, Nq <= 128, query-head pairs share a kv head
+    if (p.o_part != nullptr) {
+      if (d == 128) return launch_fwd_d<128, false, true, true>(tq, tk, tv, to, p, stream);
+      if (d == 96) return launch_fwd_d<96, false, true, true>(tq, tk, tv, to, p, stream);
+      return launch_fwd_d<64, false, true, true>(tq, tk, tv, to, p, stream);
+    }
+    if (d == 128) return launch_fwd_d<128, false, false, true>(tq, tk, tv, to, p, stream);
+    if (d == 96) return launch_fwd_d<96, false, false, true>(tq, tk, tv, to, p, stream);
+    return launch_fwd_d<64, false, false, true>(tq, tk, tv, to, p, stream);
+  }
+  if (p.o_part != nullptr) {  // partial results (dense tensors)
+    if (d == 128) return launch_fwd_d<128, false, true>(tq, tk, tv, to, p, stream);
+    if (d == 96) return launch_fwd_d<96, false, true>(tq, tk, tv, to, p, stream);
+    return launch_fwd_d<64, false, true>(tq, tk, tv, to, p, stream);
+  }
   if (d == 128)
     return vl ? launch_fwd_d<128, true>(tq, tk, tv, to, p, stream)
               : launch_fwd_d<128, false>(tq, tk, tv, to, p, stream);
@@ -561,5 +590,6 @@ cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const 
 }
 
 int fwd_rows_per_cta() { return 2 * kBM; }
+int fwd_rows_per_cta_paired() { return kBM; }
 
 }  // namespace attn_sm100

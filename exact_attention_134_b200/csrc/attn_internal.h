@@ -28,6 +28,9 @@ struct FwdParams {
   int num_splits = 1;             // key ranges per (b, h): grid z = B * num_splits
   int kv_chunk = 0;               // keys per range (a multiple of 128) when num_splits > 1
   int kv_tail = 0;                // keys after this K/V tensor in the full sequence (causal)
+  // Dense, Nq <= 128, Hq / Hkv even: a CTA's two query tiles are two query
+  // heads of one kv head (grid y = Hq / 2); num_row_blocks is then ceil(Nq / 128).
+  int pair_heads = 0;
 };
 
 // Kernel parameters of the 8-bit main kernel.
@@ -127,6 +130,7 @@ attn_status_t q8_forward_with_workspace(const void* q, const void* k, const void
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& to, const FwdParams& p, int d, cudaStream_t stream);
 int fwd_rows_per_cta();
+int fwd_rows_per_cta_paired();
 
 // O = sum_s exp(LSE_s - LSE) O_s, LSE = ln sum_s exp(LSE_s) over num_parts
 // partial results [num_parts, rows, d] fp32 / [num_parts, rows] fp32;

@@ -72,7 +72,9 @@ typedef enum {
  *   lse    device, fp32 [B, Hq, Nq]             (written)
  *   scale  softmax scale applied to Q K^T (typically 1/sqrt(d)); finite, > 0
  *   causal 0 = full attention, 1 = causal mask aligned to the bottom right
- * Allocates nothing; one kernel launch on `stream`.
+ * Allocates nothing; one kernel launch on `stream`. A CTA computes two 128-row
+ * query tiles sharing each K/V tile: 256 rows of one query head, or, when
+ * Nq <= 128 and Hq / Hkv is even, the rows of two query heads of one kv head.
  */
 ATTN_API attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                        int B, int Hq, int Hkv, int Nq, int Nkv, int d,
@@ -155,8 +157,9 @@ ATTN_API attn_status_t attn_merge_partials(const float* o_parts, const float* ls
  *               16-byte aligned, owned by the caller: the fp32 partials
  * Two launches (partials, merge). ATTN_ERR_UNSUPPORTED if B * ranges > 65535.
  */
-ATTN_API int attn_fwd_splitkv_num_splits(int B, int Hq, int Nq, int Nkv, int num_splits);
-ATTN_API size_t attn_fwd_splitkv_workspace_size(int B, int Hq, int Nq, int Nkv, int d,
+ATTN_API int attn_fwd_splitkv_num_splits(int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                                         int num_splits);
+ATTN_API size_t attn_fwd_splitkv_workspace_size(int B, int Hq, int Hkv, int Nq, int Nkv, int d,
                                                 int num_splits);
 ATTN_API attn_status_t attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
                                         float* lse, int B, int Hq, int Hkv, int Nq, int Nkv,

@@ -159,16 +159,18 @@ def test_partial_and_merge_entry_validation(lib):
 def test_splitkv_plan_and_validation(lib):
     # the automatic choice fills one wave of CTAs (at most 148 here: without a
     # GPU the library assumes 148 SMs) with ranges of at least two key tiles
-    assert attn.splitkv_num_splits(1, 32, 128, 131072) == 4      # 32 CTAs -> 4 ranges
-    assert attn.splitkv_num_splits(2, 32, 8192, 8192) == 1       # already > 148 CTAs
-    assert attn.splitkv_num_splits(1, 1, 16, 1 << 20) == 64      # capped at 64 ranges
-    assert attn.splitkv_num_splits(1, 2, 10, 300) == 1           # 3 tiles: ranges of >= 2
-    assert attn.splitkv_num_splits(1, 2, 10, 1000, 5) == 4       # 8 tiles in ranges of 2
-    assert attn.splitkv_num_splits(1, 2, 10, 1000, 100) == 8     # at most one range per tile
-    assert attn.splitkv_num_splits(0, 2, 10, 1000) == 0
-    need = lib.attn_fwd_splitkv_workspace_size(1, 32, 128, 131072, 128, 0)
-    assert need >= 4 * 32 * 128 * (128 + 1) * 4 and need % 256 == 0
-    assert lib.attn_fwd_splitkv_workspace_size(2, 32, 8192, 8192, 128, 0) == 0  # one range
+    n = attn.splitkv_num_splits
+    assert n(1, 32, 8, 128, 131072, 128) == 9     # head pairs: 16 CTAs -> 9 ranges
+    assert n(1, 32, 32, 128, 131072, 128) == 4    # one head per CTA: 32 CTAs -> 4 ranges
+    assert n(2, 32, 32, 8192, 8192, 128) == 1     # already > 148 CTAs
+    assert n(1, 1, 1, 16, 1 << 20, 128) == 64     # capped at 64 ranges
+    assert n(1, 2, 2, 10, 300, 128) == 1          # 3 tiles: ranges of >= 2
+    assert n(1, 2, 2, 10, 1000, 128, 5) == 4      # 8 tiles in ranges of 2
+    assert n(1, 2, 2, 10, 1000, 128, 100) == 8    # at most one range per tile
+    assert n(0, 2, 2, 10, 1000, 128) == 0 and n(1, 3, 2, 10, 1000, 128) == 0
+    need = lib.attn_fwd_splitkv_workspace_size(1, 32, 8, 128, 131072, 128, 0)
+    assert need >= 9 * 32 * 128 * (128 + 1) * 4 and need % 256 == 0
+    assert lib.attn_fwd_splitkv_workspace_size(2, 32, 32, 8192, 8192, 128, 0) == 0  # one range
 
     def call(ws=P, nbytes=need, d=128, B=1, S=0):
         return lib.attn_fwd_splitkv(P, P, P, P, P, B, 32, 8, 128, 131072, d, 0, 0.1, S, ws,

@@ -78,6 +78,11 @@ SMALL = [
     (1, 4, 2, 100, 333, 128, False),
     (2, 4, 1, 512, 64, 64, False),
     (1, 2, 2, 640, 1900, 128, False),
+    # Nq <= 128 with an even GQA group: two query heads per CTA
+    (2, 8, 2, 128, 1000, 128, True),
+    (1, 4, 2, 1, 513, 64, False),
+    (1, 6, 3, 77, 77, 96, True),
+    (1, 8, 1, 100, 300, 64, True),
     (1, 16, 2, 1024, 1024, 128, True),
     # head dim 96: three 32-column boxes per row
     (1, 2, 2, 256, 256, 96, False),

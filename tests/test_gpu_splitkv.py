@@ -101,6 +101,7 @@ SPLIT = [
     (1, 2, 2, 300, 1000, 96, True, 2),
     (1, 2, 2, 513, 513, 128, True, 4),      # square causal: ranges past a row's diagonal
     (1, 2, 2, 1, 777, 128, True, 0),         # one query row (decode)
+    (1, 4, 2, 64, 1500, 96, True, 3),        # head pairs, d = 96
 ]
 
 
@@ -108,7 +109,7 @@ SPLIT = [
 def test_splitkv_matches_oracle(case):
     B, Hq, Hkv, Nq, Nkv, d, causal, S = case
     q, k, v = make_qkv(B, Hq, Hkv, Nq, Nkv, d, seed=sum(case[:6]))
-    assert attn.splitkv_num_splits(B, Hq, Nq, Nkv, S) > 1
+    assert attn.splitkv_num_splits(B, Hq, Hkv, Nq, Nkv, d, S) > 1
     o, lse = attn.attn_fwd_splitkv(q.cuda(), k.cuda(), v.cuda(), causal=causal, num_splits=S)
     _status_ok()
     assert o.dtype == torch.bfloat16
