@@ -182,6 +182,14 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.num_row_blocks = (Nq + rows - 1) / rows;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
+  // Causal row blocks differ in cost: dispatch the heaviest of a group of
+  // (batch, query head) pairs first, the group's kv heads holding at most
+  // 32 MiB of K and V so that they stay in L2 while the group runs.
+  if (causal && d != 256 && !p.pair_heads && !part.o_part && p.num_row_blocks > 1) {
+    const long long kv_head_bytes = 4LL * Nkv * d;
+    const long long kv_heads = std::max(1LL, (32LL << 20) / kv_head_bytes);
+    p.lpt_group = (int)std::min((long long)B * Hq, kv_heads * (Hq / Hkv));
+  }
   p.o_part = part.o_part;
   p.num_splits = part.num_splits;
   p.kv_chunk = part.kv_chunk;

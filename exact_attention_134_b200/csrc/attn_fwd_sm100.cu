@@ -156,6 +156,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   // ---- work unit: 256 query rows of one (sequence, query head)
+  // Dense causal launches dispatch the row blocks heaviest first across
+  // groups of p.lpt_group (batch, query head) pairs (longest processing time
+  // first, within groups whose K/V stay in L2): the linear block index is
+  // remapped to (row-block rank ux, head uy, batch uz).
+  int ux = blockIdx.x, uy = blockIdx.y, uz = blockIdx.z;
+  if (!VL && !PART && p.lpt_group > 0) {
+    const long long nx = gridDim.x, nyz = (long long)gridDim.y * gridDim.z;
+    const long long lin = blockIdx.x + nx * (blockIdx.y + (long long)gridDim.y * blockIdx.z);
+    const long long per_group = nx * p.lpt_group;
+    const long long g = lin / per_group;
+    const long long first = g * p.lpt_group;  // first (head, batch) pair of the group
+    const long long n_in = min((long long)p.lpt_group, nyz - first);
+    const long long within = lin - g * per_group;
+    const long long yz = first + within % n_in;
+    ux = (int)(within / n_in);
+    uy = (int)(yz % gridDim.y);
+    uz = (int)(yz / gridDim.y);
+  }
   int Lq = p.Nq, Lk = p.Nkv, q_start = 0, k_start = 0;
   if (VL) {
     const int sq = blockIdx.z;
@@ -171,10 +189,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kUnitRows = PAIR ? kBM : 2 * kBM;  // query rows of a work unit
   constexpr int kTileRowStep = PAIR ? 0 : kBM;    // first row of tile 1 - of tile 0
   const int nrb = (Lq + kUnitRows - 1) / kUnitRows;
-  if ((int)blockIdx.x >= nrb) return;  // this sequence has fewer rows (the whole CTA leaves)
-  const int row_block = p.causal ? (nrb - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-  const int hq = PAIR ? 2 * (int)blockIdx.y : (int)blockIdx.y;  // query head of tile 0
-  const int b = VL ? 0 : (PART ? (int)blockIdx.z / p.num_splits : (int)blockIdx.z);
+  if (ux >= nrb) return;  // this sequence has fewer rows (the whole CTA leaves)
+  const int row_block = p.causal ? (nrb - 1 - ux) : ux;
+  const int hq = PAIR ? 2 * uy : uy;  // query head of tile 0
+  const int b = VL ? 0 : (PART ? uz / p.num_splits : uz);
   const int hk = hq / (p.Hq / p.Hkv);
   const int q0 = row_block * kUnitRows;  // first query row of the unit, within its sequence
   const int bh_q = b * p.Hq + hq;        // (tile 1: bh_q + 1 when PAIR)

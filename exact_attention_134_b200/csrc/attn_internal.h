@@ -31,6 +31,9 @@ struct FwdParams {
   // Dense, Nq <= 128, Hq / Hkv even: a CTA's two query tiles are two query
   // heads of one kv head (grid y = Hq / 2); num_row_blocks is then ceil(Nq / 128).
   int pair_heads = 0;
+  // Dense causal, one head per CTA: dispatch order groups (0 = the grid's own
+  // order, each head's row blocks heaviest first). See attn_fwd_bf16_kernel.
+  int lpt_group = 0;
 };
 
 // Kernel parameters of the 8-bit main kernel.
