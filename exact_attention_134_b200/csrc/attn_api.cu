@@ -447,6 +447,11 @@ attn_status_t run_bwd(const void* q, const void* k, const void* v, const void* o
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
+  if (causal && !vl && Nkv > 128) {
+    // a group's Q, dO (bf16) and dQ accumulator (fp32) within 32 MiB
+    const long long per_kv_head = 8LL * Nq * d * (Hq / Hkv);
+    p.lpt_group = (int)std::min((long long)B * Hkv, std::max(1LL, (32LL << 20) / per_kv_head));
+  }
   L.post.dq_acc = acc;
   L.post.dq = dq;
   L.post.cu_q = cu_q;

@@ -212,9 +212,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   // ---- work unit: 128 keys of one (batch, kv head)
-  const int kb = blockIdx.x;
-  const int hk = blockIdx.y;
-  const int b = blockIdx.z;  // batch entry, or sequence (VL)
+  // Dense causal launches dispatch key blocks heaviest first (the first keys
+  // are seen by the most queries) across groups of p.lpt_group (kv head,
+  // batch) pairs whose Q, dO and dQ accumulator stay in L2.
+  int kb = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;  // b: batch entry, or sequence (VL)
+  if (!VL && p.lpt_group > 0) {
+    const long long nx = gridDim.x, nyz = (long long)gridDim.y * gridDim.z;
+    const long long lin = blockIdx.x + nx * (blockIdx.y + (long long)gridDim.y * blockIdx.z);
+    const long long per_group = nx * p.lpt_group;
+    const long long g = lin / per_group;
+    const long long first = g * p.lpt_group;
+    const long long n_in = min((long long)p.lpt_group, nyz - first);
+    const long long within = lin - g * per_group;
+    const long long yz = first + within % n_in;
+    kb = (int)(within / n_in);
+    hk = (int)(yz % gridDim.y);
+    b = (int)(yz / gridDim.y);
+  }
   const int G = p.Hq / p.Hkv;
   const int k0 = kb * kBK;
   int Lq = p.Nq, Lk = p.Nkv, q_start = 0, k_start = 0;

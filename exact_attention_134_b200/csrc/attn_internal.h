@@ -89,6 +89,9 @@ struct BwdParams {
   float scale;
   float scale_log2;
   unsigned long long timeout_ns;
+  // Dense causal: dispatch order groups of (batch, kv head) pairs, key blocks
+  // heaviest first across a group (0 = the grid's own order).
+  int lpt_group;
 };
 
 struct BwdPreParams {
