@@ -185,7 +185,7 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   // Causal row blocks differ in cost: dispatch the heaviest of a group of
   // (batch, query head) pairs first, the group's kv heads holding at most
   // 32 MiB of K and V so that they stay in L2 while the group runs.
-  if (causal && d != 256 && !p.pair_heads && !part.o_part && p.num_row_blocks > 1) {
+  if (causal && !p.pair_heads && !part.o_part && Nq > 128) {
     const long long kv_head_bytes = 4LL * Nkv * d;
     const long long kv_heads = std::max(1LL, (32LL << 20) / kv_head_bytes);
     p.lpt_group = (int)std::min((long long)B * Hq, kv_heads * (Hq / Hkv));
@@ -310,6 +310,10 @@ attn_status_t run_q8(const void* q, const void* k, const void* v, void* o, float
   p.num_row_blocks = (Nq + 255) / 256;
   p.nqb = (Nq + 127) / 128;
   p.nkb = (Nkv + 127) / 128;
+  if (causal && Nq > 256) {  // as the bf16 forward, for 8-bit K and V
+    const long long kv_heads = std::max(1LL, (32LL << 20) / (2LL * Nkv * d));
+    p.lpt_group = (int)std::min((long long)B * Hq, kv_heads * (Hq / Hkv));
+  }
   p.scale_log2 = scale * 1.4426950408889634f;
   p.scale = scale;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();

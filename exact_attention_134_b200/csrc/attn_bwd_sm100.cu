@@ -215,20 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Dense causal launches dispatch key blocks heaviest first (the first keys
   // are seen by the most queries) across groups of p.lpt_group (kv head,
   // batch) pairs whose Q, dO and dQ accumulator stay in L2.
-  int kb = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;  // b: batch entry, or sequence (VL)
-  if (!VL && p.lpt_group > 0) {
-    const long long nx = gridDim.x, nyz = (long long)gridDim.y * gridDim.z;
-    const long long lin = blockIdx.x + nx * (blockIdx.y + (long long)gridDim.y * blockIdx.z);
-    const long long per_group = nx * p.lpt_group;
-    const long long g = lin / per_group;
-    const long long first = g * p.lpt_group;
-    const long long n_in = min((long long)p.lpt_group, nyz - first);
-    const long long within = lin - g * per_group;
-    const long long yz = first + within % n_in;
-    kb = (int)(within / n_in);
-    hk = (int)(yz % gridDim.y);
-    b = (int)(yz / gridDim.y);
-  }
+  int kb, hk, b;  // b: batch entry, or sequence (VL)
+  grouped_heavy_first(VL ? 0 : p.lpt_group, kb, hk, b);
   const int G = p.Hq / p.Hkv;
   const int k0 = kb * kBK;
   int Lq = p.Nq, Lk = p.Nkv, q_start = 0, k_start = 0;

@@ -107,9 +107,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- work unit: 128 query rows of one (batch, query head)
   const int nrb = (p.Nq + kBM - 1) / kBM;
-  const int row_block = p.causal ? (nrb - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-  const int hq = blockIdx.y;
-  const int b = blockIdx.z;
+  // causal: row blocks heaviest first across groups of heads (see grouped_heavy_first)
+  int ux, hq, b;
+  grouped_heavy_first(p.lpt_group, ux, hq, b);
+  const int row_block = p.causal ? (nrb - 1 - ux) : ux;
   const int hk = hq / (p.Hq / p.Hkv);
   const int q0 = row_block * kBM;
   const int bh_q = b * p.Hq + hq;

@@ -157,23 +157,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- work unit: 256 query rows of one (sequence, query head)
   // Dense causal launches dispatch the row blocks heaviest first across
-  // groups of p.lpt_group (batch, query head) pairs (longest processing time
-  // first, within groups whose K/V stay in L2): the linear block index is
-  // remapped to (row-block rank ux, head uy, batch uz).
-  int ux = blockIdx.x, uy = blockIdx.y, uz = blockIdx.z;
-  if (!VL && !PART && p.lpt_group > 0) {
-    const long long nx = gridDim.x, nyz = (long long)gridDim.y * gridDim.z;
-    const long long lin = blockIdx.x + nx * (blockIdx.y + (long long)gridDim.y * blockIdx.z);
-    const long long per_group = nx * p.lpt_group;
-    const long long g = lin / per_group;
-    const long long first = g * p.lpt_group;  // first (head, batch) pair of the group
-    const long long n_in = min((long long)p.lpt_group, nyz - first);
-    const long long within = lin - g * per_group;
-    const long long yz = first + within % n_in;
-    ux = (int)(within / n_in);
-    uy = (int)(yz % gridDim.y);
-    uz = (int)(yz / gridDim.y);
-  }
+  // groups of p.lpt_group (batch, query head) pairs whose K/V stay in L2:
+  // (row-block rank ux, head uy, batch uz).
+  int ux, uy, uz;
+  grouped_heavy_first((!VL && !PART) ? p.lpt_group : 0, ux, uy, uz);
   int Lq = p.Nq, Lk = p.Nkv, q_start = 0, k_start = 0;
   if (VL) {
     const int sq = blockIdx.z;

@@ -48,6 +48,7 @@ struct Q8Params {
   int causal;
   int num_row_blocks;
   int nqb, nkb;                   // 128-token blocks of Q and K/V
+  int lpt_group;                  // causal dispatch order groups (0 = grid order)
   float scale_log2;               // scale * log2(e)
   float scale;
   unsigned long long timeout_ns;

@@ -365,8 +365,10 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int row_block = p.causal ? (p.num_row_blocks - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-  const int hq = blockIdx.y, b = blockIdx.z;
+  // causal: row blocks heaviest first across groups of heads (see grouped_heavy_first)
+  int ux, hq, b;
+  grouped_heavy_first(p.lpt_group, ux, hq, b);
+  const int row_block = p.causal ? (p.num_row_blocks - 1 - ux) : ux;
   const int hk = hq / (p.Hq / p.Hkv);
   const int q0 = row_block * 2 * kTok;
   const int bh_q = b * p.Hq + hq;

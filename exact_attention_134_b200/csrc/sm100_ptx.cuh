@@ -98,6 +98,32 @@ __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity,
   return false;
 }
 
+// ---------------------------------------------------------------- work order
+// Longest processing time first, within groups: the grid's x index is a
+// block's cost rank within its (y, z) pair (0 = heaviest); blocks are taken
+// in linear order, so remapping the linear index makes the hardware dispatch
+// the heaviest blocks of `group` consecutive (y, z) pairs first, then the
+// next heaviest of the same pairs, and so on, one group after another (a
+// group sized so that its pairs' data stay in L2). group <= 0 keeps the
+// grid's own order (every pair's blocks heaviest first, pair after pair).
+__device__ __forceinline__ void grouped_heavy_first(int group, int& ux, int& uy, int& uz) {
+  ux = blockIdx.x;
+  uy = blockIdx.y;
+  uz = blockIdx.z;
+  if (group <= 0) return;
+  const long long nx = gridDim.x, nyz = (long long)gridDim.y * gridDim.z;
+  const long long lin = blockIdx.x + nx * (blockIdx.y + (long long)gridDim.y * blockIdx.z);
+  const long long per_group = nx * group;
+  const long long g = lin / per_group;
+  const long long first = g * group;  // first (y, z) pair of the group
+  const long long n_in = min((long long)group, nyz - first);
+  const long long within = lin - g * per_group;
+  const long long yz = first + within % n_in;
+  ux = (int)(within / n_in);
+  uy = (int)(yz % gridDim.y);
+  uz = (int)(yz / gridDim.y);
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
