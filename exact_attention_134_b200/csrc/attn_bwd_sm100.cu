@@ -212,11 +212,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   // ---- work unit: 128 keys of one (batch, kv head)
-  // Dense causal launches dispatch key blocks heaviest first (the first keys
-  // are seen by the most queries) across groups of p.lpt_group (kv head,
-  // batch) pairs whose Q, dO and dQ accumulator stay in L2.
+  // Causal launches dispatch key blocks heaviest first (the first keys are
+  // seen by the most queries) across groups of p.lpt_group (kv head, batch or
+  // sequence) pairs whose Q, dO and dQ accumulator stay in L2.
   int kb, hk, b;  // b: batch entry, or sequence (VL)
-  grouped_heavy_first(VL ? 0 : p.lpt_group, kb, hk, b);
+  grouped_heavy_first(p.lpt_group, kb, hk, b);
   const int G = p.Hq / p.Hkv;
   const int k0 = kb * kBK;
   int Lq = p.Nq, Lk = p.Nkv, q_start = 0, k_start = 0;
