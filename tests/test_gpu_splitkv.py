@@ -159,3 +159,29 @@ def test_splitkv_long_cache_sampled_rows():
     lg = np.take_along_axis(lse.cpu().numpy().astype(np.float64), rows, axis=2)
     d = np.abs(og - O)
     assert d.max() <= MAX_TOL and d.mean() <= MEAN_TOL and np.abs(lg - L).max() <= LSE_TOL
+
+
+def test_kv_sharded_module_single_rank_nccl():
+    """kv_shard.attention_kv_sharded through its default path (attn_fwd_partial,
+    an NCCL all-gather, merge_partials) in a one-rank process group: the
+    product code of the key-sharded forward on the GPU; its multi-rank host
+    logic is tested with gloo ranks on the CPU."""
+    import socket
+    import torch.distributed as dist
+    from exact_attention_134_b200.kv_shard import attention_kv_sharded
+    if dist.is_initialized():
+        pytest.skip("a process group already exists")
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device("cuda:0"))
+    try:
+        B, Hq, Hkv, Nq, Nkv, d = 1, 4, 2, 200, 900, 128
+        q, k, v = make_qkv(B, Hq, Hkv, Nq, Nkv, d, seed=91)
+        o, lse = attention_kv_sharded(q.cuda(), k.cuda(), v.cuda(), Nkv, causal=True)
+        _status_ok()
+        O, L = oracle.attention_fp64(bf16_bits(q), bf16_bits(k), bf16_bits(v), True, 1 / math.sqrt(d))
+        _check(o, lse, O, L)
+    finally:
+        dist.destroy_process_group()
