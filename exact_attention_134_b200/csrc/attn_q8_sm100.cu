@@ -35,7 +35,9 @@ constexpr int kQ8Threads = 320;
 #ifndef ATTN_Q8_EMU
 #define ATTN_Q8_EMU 0
 #endif
-// 1: half of the exponentials of unmasked tiles use the FMA-pipe polynomial
+// Build option, off by default: 1 puts half of the exponentials of unmasked
+// tiles on the FMA pipe (exp2_poly2). On the B200 it measured slower: the
+// softmax step is bound by its dependency chain, not by the MUFU unit alone.
 constexpr bool kQ8EmuHalf = ATTN_Q8_EMU != 0;
 constexpr int kTok = 128;         // tokens per quantisation block == MMA tile rows
 constexpr int kPrepThreads = 256;
