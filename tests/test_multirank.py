@@ -166,3 +166,39 @@ def test_kv_sharded_three_ranks_gloo(causal):
     for r in range(world):
         o, lse = res[r]
         assert np.abs(o - O).max() < 1e-12 and np.abs(lse - L).max() < 1e-12
+
+
+def _kv_errors_worker(port, out):
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    import torch.distributed as dist
+    from exact_attention_134_b200.kv_shard import attention_kv_sharded
+    dist.init_process_group("gloo", rank=0, world_size=1)
+    q = torch.zeros(1, 2, 4, 8)
+    k = torch.zeros(1, 2, 5, 8)
+    msgs = []
+    for n_keys, kk in ((6, k), (0, k[:, :, :0])):
+        try:
+            attention_kv_sharded(q, kk, kk, n_keys, partial_fn=lambda *a, **kw: None,
+                                 merge_fn=lambda *a: None)
+            msgs.append("no error")
+        except ValueError as e:
+            msgs.append(str(e))
+    out[0] = msgs
+    dist.destroy_process_group()
+
+
+def test_kv_sharded_rejects_wrong_shards():
+    """A rank whose K/V do not hold exactly its range, or a key count below the
+    number of ranks, is refused before any kernel or exchange runs."""
+    if torch.cuda.is_available():
+        pytest.skip("CPU/gloo test")
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        p = ctx.Process(target=_kv_errors_worker, args=(_free_port(), out))
+        p.start()
+        p.join(120)
+        assert p.exitcode == 0
+        msgs = out[0]
+    assert "must hold keys [0, 6) of 6" in msgs[0]
+    assert "at least one key" in msgs[1]
