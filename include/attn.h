@@ -1,5 +1,6 @@
 /*
- * attn.h — C ABI of the B200 (sm_100a) fused exact-attention forward.
+ * attn.h — C ABI of the B200 (sm_100a) fused exact attention: forward (bf16,
+ * 8-bit, packed sequences, key-range partials and their merge) and backward.
  *
  * Operation (the definition on "FlashAttention (TR)", systems-analysis.info,
  * section "Standart Attention Mekanizmasının Sorunları"):
@@ -24,7 +25,8 @@
  *   - Head dim d is 64, 96 or 128; attn_fwd and attn_fwd_host also take 256
  *     (the "FlashAttention-2 (2023)" section's largest head dimension; its own
  *     kernel: one query tile per CTA, Q held in tensor memory); the 8-bit
- *     entry points take 64 or 128, the backward 64, 96 or 128.
+ *     entry points take 64 or 128; the backward, attn_fwd_partial and
+ *     attn_fwd_splitkv 64, 96 or 128; attn_merge_partials 64, 96, 128, 256.
  *   - Ownership: the caller owns every buffer; device pointers must stay valid
  *     until the work queued on `stream` has finished. The library allocates no
  *     device memory. `stream` is a cudaStream_t (0 = legacy default stream).
