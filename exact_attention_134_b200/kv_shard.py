@@ -13,7 +13,8 @@ Softmax Hesaplama", applied to whole key ranges — exact in real arithmetic.
 The causal mask stays the full sequence's (bottom-right aligned): a rank
 passes the number of keys held by the ranks after it as ``kv_tail``.
 
-The exchange is one all-gather of B*Hq*Nq*(d+1) fp32 values per rank.
+The exchange is two all-gathers (O and LSE) of B*Hq*Nq*(d+1) fp32 values
+per rank in all.
 """
 from __future__ import annotations
 
