@@ -55,6 +55,7 @@ PARTIAL = [
     (2, 2, 1, 129, 64, 700, 0, 64, True),       # the last range of a prefill with a cache
     (1, 2, 2, 77, 1000, 260, 37, 96, True),
     (1, 4, 4, 256, 256, 512, 256, 128, False),
+    (1, 4, 2, 100, 300, 500, 200, 128, True),   # head pairs (Nq <= 128, even group)
 ]
 
 
