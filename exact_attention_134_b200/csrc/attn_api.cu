@@ -494,6 +494,8 @@ attn_status_t q8_forward_with_workspace(const void* q, const void* k, const void
 
 }  // namespace attn_sm100
 
+namespace {
+
 // Split of the keys for attn_fwd_splitkv: num_splits <= 0 picks as many ranges
 // as fill one wave of CTAs (one per SM, the forward kernel's occupancy) without
 // starting a second, partly empty one; ranges hold at least two 128-key tiles.
@@ -534,6 +536,8 @@ SplitLayout splitkv_layout(int splits, int B, int Hq, int Nq, int d) {
   const size_t lse_off = round_up(rows * d * 4, 256);
   return {lse_off, round_up(lse_off + rows * 4, 256)};
 }
+
+}  // namespace
 
 extern "C" {
 
