@@ -18,7 +18,6 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -428,7 +427,6 @@ def bench_e2e(w: Workload, steps: int, warmup: int, world: int, rank: int, lib_m
 def cpu_baseline(w: Workload, q, k, v, budget_s: float = 12.0):
     """The fp64 oracle, as it stands, on the host cores over a bounded sample:
     whole (batch, head) pairs in order until ~budget_s of CPU work."""
-    import numpy as np
     import oracle
     cores = len(os.sched_getaffinity(0))
     qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)

@@ -14,7 +14,7 @@ import torch
 
 import exact_attention_134_b200 as attn
 import oracle
-from synthetic import WORKLOADS, bf16_bits, make_qkv, make_workload, sample_rows
+from synthetic import WORKLOADS, bf16_bits, make_qkv, sample_rows
 
 pytestmark = pytest.mark.gpu
 
