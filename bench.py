@@ -266,14 +266,22 @@ def bench_workload(w: Workload, steps: int, warmup: int, world: int, rank: int, 
     res = {"total_ms": total_ms, "times": times, "l2": l2_mode, "inputs": (q, k, v),
            "flops": w.flops}
     if graph:
+        # every rank takes part in both reductions, whatever happened locally
+        err, local_ms = None, 0.0
         try:
             gt = time_graph_replays(step, steps, flush)
             st, where = lib_mod.get_status()
             if st != 0:
                 raise RuntimeError(f"device status {st} at {where:#x}")
-            res["graph_total_ms"] = _max_over_ranks(sum(gt), world)
+            local_ms = sum(gt)
         except Exception as e:  # noqa: BLE001 - reported in the JSON line, eager time stands
-            res["graph_error"] = f"{type(e).__name__}: {e}"[:200]
+            err = f"{type(e).__name__}: {e}"[:200]
+        any_err = _max_over_ranks(1.0 if err else 0.0, world)
+        graph_ms = _max_over_ranks(local_ms, world)
+        if any_err == 0.0:
+            res["graph_total_ms"] = graph_ms
+        else:
+            res["graph_error"] = err or "graph timing failed on another rank"
     return res
 
 
