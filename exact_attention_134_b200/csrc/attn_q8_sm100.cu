@@ -14,9 +14,11 @@
 //                 qk_i = q_i . kbar (to undo the smoothing shift in LSE);
 //                 K - kbar -> INT8 per 128-token block; V / sv -> e4m3
 //   4. main       the fused forward: S = Q8 K8^T (kind::i8, s32 in TMEM),
-//                 online softmax on s * sq * sk * scale, P -> e4m3(p * 448)
+//                 online softmax on s * sq * sk * scale with a reference
+//                 maximum that may lag the row maximum by up to 2^4 (so O
+//                 is rescaled only rarely), P -> e4m3(p * 448 / 16) (p <= 16)
 //                 written back to TMEM, O += P8 V8 (kind::f8f6f4, fp32 in
-//                 TMEM), O = O * sv / (448 l), LSE += scale * qk.
+//                 TMEM), O = O * sv / (28 l), LSE += scale * qk.
 // Every quantisation decision (scale, code) is taken in fp32 with correctly
 // rounded division and round-half-even, so the codes are reproducible.
 #include <cuda.h>
@@ -547,9 +549,13 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     // a tile wholly past Nq has no scale; its rows are computed but never stored
     const float sq_t = qtile < p.nqb ? p.sq[(size_t)bh_q * p.nqb + qtile] : 1.0f;
     const float kLog2_448 = 8.807354922057604f;  // log2(448)
+    // the reference maximum may lag the row maximum by up to kLag (log2 units):
+    // P is encoded as 2^(t - m_ref) * 448 * 2^-kLag <= 448, and O is rescaled
+    // only when a tile's maximum exceeds m_ref + kLag
+    constexpr float kLag = 4.0f;
 
-    float m_run = -INFINITY;  // running maximum of scale*log2(e)*S (exact: rescale on every increase)
-    float l_run = 0.0f;       // sum of 448 * 2^(. - m_run)
+    float m_run = -INFINITY;  // reference maximum of scale*log2(e)*S: within kLag below the row maximum
+    float l_run = 0.0f;       // sum of 448 * 2^-kLag * 2^(. - m_run)
     bool ok = true;
     int j = 0;
     for (; j < n_tiles; ++j) {
@@ -595,13 +601,13 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
       // f > 0 (all scales positive), so the max of s*f is f * max(s)
       const float m_tile = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * f;
       float alpha = 1.0f;
-      if (m_tile > m_run) {
+      if (m_tile > m_run + kLag) {
         alpha = ex2_approx(m_run - m_tile);
         m_run = m_tile;
       }
       const float mb = (m_run == -INFINITY) ? 0.0f : m_run;
-      // p448 = 448 * 2^(s*f - m) = 2^(s*f - m + log2 448)
-      const float2 slope = make_float2(f, f), bias = make_float2(kLog2_448 - mb, kLog2_448 - mb);
+      // p = 448 * 2^-kLag * 2^(s*f - m) = 2^(s*f - m + log2 448 - kLag) <= 448
+      const float2 slope = make_float2(f, f), bias = make_float2(kLog2_448 - kLag - mb, kLog2_448 - kLag - mb);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
 #pragma unroll
@@ -675,8 +681,8 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
       fence_proxy_async_smem();
       mbar_arrive(bar(Q8Bar::kEpi + t));
       if (row < p.Nq) {
-        // l_run carries the factor 448, which O's numerator also carries
-        const float lse2 = m_run + log2f(l_run) - kLog2_448;
+        // l_run carries the factor 448 * 2^-kLag, which O's numerator also carries
+        const float lse2 = m_run + log2f(l_run) - (kLog2_448 - kLag);
         p.lse[(size_t)bh_q * p.Nq + row] =
             lse2 * 0.69314718055994530942f + p.scale * p.qk[(size_t)bh_q * p.Nq + row];
       }
