@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     mbar_init(bar(Q8Bar::kQFull), 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(Q8Bar::kSFull + t), 1);
-      mbar_init(bar(Q8Bar::kPFull + t), 128);
+      mbar_init(bar(Q8Bar::kPFull + t), 4);  // one arrival per softmax warp
       mbar_init(bar(Q8Bar::kEpi + t), 128);
     }
     mbar_init(bar(Q8Bar::kOFinal), 1);
@@ -558,7 +558,12 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     float l_run = 0.0f;       // sum of 448 * 2^-kLag * 2^(. - m_run)
     bool ok = true;
     int j = 0;
+    // the K block scale of the next tile is loaded a step ahead (off the chain)
+    const float* const sk_row = p.sk + (size_t)bh_kv * p.nkb;
+    float sk_next = __ldg(sk_row);
     for (; j < n_tiles; ++j) {
+      const float sk_j = sk_next;
+      if (j + 1 < n_tiles) sk_next = __ldg(sk_row + j + 1);
       ok = q8_warp_all(bounded_wait(bar(Q8Bar::kSFull + t), j & 1, abort_flag, budget));
       if (!ok) break;
       tc_fence_after();
@@ -567,7 +572,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
       for (int c = 0; c < 4; ++c)
         tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
       tmem_wait_ld();
-      const float f = sq_t * p.sk[(size_t)bh_kv * p.nkb + j] * p.scale_log2;
+      const float f = sq_t * sk_j * p.scale_log2;
       // s32 -> fp32 without the conversion unit: |s| <= 127 * 127 * d < 2^22, so
       // the bits of (s + 0x4B400000) are the float 1.5 * 2^23 + s exactly
       // (the e4m3 MMA already accumulates in fp32)
@@ -646,7 +651,8 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
       l_run = l_run * alpha + row_sum;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(Q8Bar::kPFull + t));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(Q8Bar::kPFull + t));
     }
 
     if (ok) ok = q8_warp_all(bounded_wait(bar(Q8Bar::kOFinal), 0, abort_flag, budget));
