@@ -34,13 +34,12 @@ namespace attn_sm100 {
 namespace {
 
 constexpr int kQ8Threads = 320;
-#ifndef ATTN_Q8_EMU
-#define ATTN_Q8_EMU 0
-#endif
-// Build option, off by default: 1 puts half of the exponentials of unmasked
-// tiles on the FMA pipe (exp2_poly2). On the B200 it measured slower: the
-// softmax step is bound by its dependency chain, not by the MUFU unit alone.
-constexpr bool kQ8EmuHalf = ATTN_Q8_EMU != 0;
+// Exponentials of the softmax: of every 8 groups of 4, the first kPolyOf8 are
+// evaluated by exp2_poly2 on the FMA pipe, the rest by ex2.approx. The 8-bit
+// softmax's e4m3 packing competes with ex2 for issue; moving 3/8 of the
+// exponentials off it shortened the loop by ~9 % in a register-only B200
+// measurement of the same instruction mix (1/8 and 1/2 were slower).
+constexpr int kPolyOf8 = 3;
 constexpr int kTok = 128;         // tokens per quantisation block == MMA tile rows
 constexpr int kPrepThreads = 256;
 
@@ -573,18 +572,15 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
         tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
       tmem_wait_ld();
       const float f = sq_t * sk_j * p.scale_log2;
-      // s32 -> fp32 without the conversion unit: |s| <= 127 * 127 * d < 2^22, so
-      // the bits of (s + 0x4B400000) are the float 1.5 * 2^23 + s exactly
-      // (the e4m3 MMA already accumulates in fp32)
+      // s32 -> fp32 without a conversion instruction: |s| <= 127 * 127 * d < 2^22,
+      // so the bits of (s + 0x4B400000) are the float M + s exactly, M = 1.5 * 2^23.
+      // Those floats order like s (same binade), so the row maximum is taken on
+      // them, and M * f is folded into the exponent's bias below. (The e4m3 MMA
+      // already accumulates in fp32: kOff = 0.)
       constexpr float kMagic = 12582912.0f;
+      constexpr float kOff = F8 ? 0.0f : kMagic;
 #pragma unroll
-      for (int c = 0; c < (F8 ? 0 : kTok); c += 2) {
-        const float2 v = add2(make_float2(__uint_as_float(sr[c] + 0x4B400000u),
-                                          __uint_as_float(sr[c + 1] + 0x4B400000u)),
-                              make_float2(-kMagic, -kMagic));
-        sr[c] = __float_as_uint(v.x);
-        sr[c + 1] = __float_as_uint(v.y);
-      }
+      for (int c = 0; c < (F8 ? 0 : kTok); ++c) sr[c] += 0x4B400000u;
       const int kv0 = j * kTok;
       const bool tile_masked =
           (kv0 + kTok > p.Nkv) || (p.causal && kv0 + kTok - 1 > q0 + t * kTok + diag);
@@ -603,16 +599,19 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
         mx2 = fmax3(mx2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
         mx3 = fmax3(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
       }
-      // f > 0 (all scales positive), so the max of s*f is f * max(s)
-      const float m_tile = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * f;
+      // f > 0 (all scales positive), so the max of s*f is f * max(s); M + max(s) - M is exact
+      const float m_tile = (fmax3(mx0, mx1, fmaxf(mx2, mx3)) - kOff) * f;
       float alpha = 1.0f;
       if (m_tile > m_run + kLag) {
         alpha = ex2_approx(m_run - m_tile);
         m_run = m_tile;
       }
       const float mb = (m_run == -INFINITY) ? 0.0f : m_run;
-      // p = 448 * 2^-kLag * 2^(s*f - m) = 2^(s*f - m + log2 448 - kLag) <= 448
-      const float2 slope = make_float2(f, f), bias = make_float2(kLog2_448 - kLag - mb, kLog2_448 - kLag - mb);
+      // p = 448 * 2^-kLag * 2^(s*f - m) = 2^(s*f - m + log2 448 - kLag) <= 448, evaluated
+      // as (M + s) * f + (log2 448 - kLag - m - M * f): the bias is rounded once, by at
+      // most half an ulp of M * f <= 0.75 f, i.e. below one unit of the integer score
+      const float b0 = fmaf(-kOff, f, kLog2_448 - kLag - mb);
+      const float2 slope = make_float2(f, f), bias = make_float2(b0, b0);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
 #pragma unroll
@@ -622,8 +621,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
         const float2 x1 = fma2(make_float2(__uint_as_float(sr[4 * qd + 2]), __uint_as_float(sr[4 * qd + 3])),
                                slope, bias);
         float2 e0, e1;
-        if (kQ8EmuHalf && !tile_masked && (qd & 1)) {
-          // half of the exponentials of unmasked tiles run on the FMA pipe
+        if ((qd & 7) < kPolyOf8) {  // arguments <= log2 448; masked ones (-inf) give ~2^-125
           e0 = exp2_poly2(x0);
           e1 = exp2_poly2(x1);
         } else {

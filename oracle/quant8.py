@@ -161,22 +161,51 @@ def q_dot_kbar(q_bits: np.ndarray, kbar: np.ndarray, Hkv: int) -> np.ndarray:
 # --------------------------------------------------------------------------
 # One-shot quantised attention built from the steps above
 # --------------------------------------------------------------------------
-def sage8_attention_fp64(q_bits, k_bits, v_bits, causal: bool, scale: float, rows=None):
-    """Quantised attention with every quantised operand taken from the steps
-    above and every other operation in float64; P is encoded relative to the
-    exact row maximum. Returns (O, LSE) float64 like ``attention_fp64``.
+def quantised_operands(q_bits, k_bits, v_bits, qk_format: str = "int8"):
+    """The operands each 8-bit method feeds its two GEMMs, from the steps above.
 
-    This is the 8-bit method's own result without online rescaling; the GPU's
-    8-bit path encodes P relative to a running maximum, so the two agree only
-    within the quantisation error, not bit for bit.
+    qk_format "int8": SageAttention's INT8 Q and mean-smoothed K (one scale per
+    128-token block), with qk = q . kbar to undo the smoothing in LSE.
+    qk_format "fp8" : e4m3 Q and K with one scale per 128-token block and no
+    smoothing (block-wise dynamic scaling in the FlashAttention-3 manner); qk = 0.
+    Both: V as e4m3 with one scale per (batch, kv head, channel).
+
+    Returns a dict of float64 arrays: qd [B,Hq,Nq,d] and kd [B,Hkv,Nkv,d] (the
+    dequantised Q and K), vd (dequantised V), qk [B,Hq,Nq], and the raw codes
+    and scales (q8, sq, k8, sk, v8, sv).
     """
     B, Hq, Nq, d = q_bits.shape
     Hkv, Nkv = k_bits.shape[1], k_bits.shape[2]
-    kbar = k_channel_mean(k_bits)
-    q8, sq = quant_int8_blocks(widen_bf16(q_bits).astype(np.float32))
-    k8, sk = quant_int8_blocks(smooth_k(k_bits, kbar))
     v8, sv = quant_v_fp8(v_bits)
-    qk = q_dot_kbar(q_bits, kbar, Hkv)
+    if qk_format == "int8":
+        kbar = k_channel_mean(k_bits)
+        q8, sq = quant_int8_blocks(widen_bf16(q_bits).astype(np.float32))
+        k8, sk = quant_int8_blocks(smooth_k(k_bits, kbar))
+        qd = q8.astype(np.float64) * np.repeat(sq, BLOCK, axis=2)[:, :, :Nq, None].astype(np.float64)
+        kd = k8.astype(np.float64) * np.repeat(sk, BLOCK, axis=2)[:, :, :Nkv, None].astype(np.float64)
+        qk = q_dot_kbar(q_bits, kbar, Hkv)
+    elif qk_format == "fp8":
+        q8, sq = quant_e4m3_blocks(widen_bf16(q_bits).astype(np.float32))
+        k8, sk = quant_e4m3_blocks(widen_bf16(k_bits).astype(np.float32))
+        qd = e4m3_decode(q8) * np.repeat(sq, BLOCK, axis=2)[:, :, :Nq, None].astype(np.float64)
+        kd = e4m3_decode(k8) * np.repeat(sk, BLOCK, axis=2)[:, :, :Nkv, None].astype(np.float64)
+        qk = np.zeros((B, Hq, Nq))
+    else:
+        raise ValueError("qk_format must be 'int8' or 'fp8'")
+    vd = e4m3_decode(v8) * sv[:, :, None, :].astype(np.float64)
+    return {"qd": qd, "kd": kd, "vd": vd, "qk": qk, "q8": q8, "sq": sq, "k8": k8, "sk": sk,
+            "v8": v8, "sv": sv}
+
+
+def _one_shot(ops, v_exact, causal: bool, scale: float, rows, quantise_pv: bool,
+              p_scale: float):
+    """softmax of the dequantised scores, then P V, one (batch, query head) at a
+    time. With quantise_pv, P is encoded as e4m3(p * p_scale) with p relative to
+    the exact row maximum and V is the dequantised e4m3 V; without it, P and V
+    are exact (only the scores carry the 8-bit error)."""
+    qd, kd = ops["qd"], ops["kd"]
+    B, Hq, Nq, d = qd.shape
+    Hkv, Nkv = kd.shape[1], kd.shape[2]
     R = Nq if rows is None else rows.shape[-1]
     O = np.empty((B, Hq, R, d))
     L = np.empty((B, Hq, R))
@@ -184,49 +213,65 @@ def sage8_attention_fp64(q_bits, k_bits, v_bits, causal: bool, scale: float, row
         for h in range(Hq):
             hk = _kv_head(h, Hq, Hkv)
             idx = np.arange(Nq) if rows is None else rows[b, h]
-            qi = q8[b, h, idx].astype(np.float64)
-            S = qi @ k8[b, hk].astype(np.float64).T
-            S *= sq[b, h, idx // BLOCK][:, None].astype(np.float64)
-            S *= sk[b, hk, np.arange(Nkv) // BLOCK][None, :].astype(np.float64)
-            S *= scale
-            if causal:
-                S = np.where(np.arange(Nkv)[None, :] <= idx[:, None], S, -np.inf)
+            S = scale * (qd[b, h, idx] @ kd[b, hk].T)
+            if causal:   # bottom-right aligned, as the exact definition
+                S = np.where(np.arange(Nkv)[None, :] <= idx[:, None] + (Nkv - Nq), S, -np.inf)
             m = S.max(axis=1)
+            empty = np.isinf(m)                     # rows that see no key
+            m = np.where(empty, 0.0, m)
             E = np.exp(S - m[:, None])
             l = E.sum(axis=1)
-            P8 = e4m3_decode(e4m3_encode((E * E4M3_MAX).astype(np.float32)))
-            Vd = e4m3_decode(v8[b, hk]) * sv[b, hk][None, :].astype(np.float64)
-            O[b, h] = (P8 @ Vd) / (E4M3_MAX * l[:, None])
-            L[b, h] = m + np.log(l) + scale * qk[b, h, idx]
+            ls = np.where(empty, 1.0, l)
+            if quantise_pv:
+                P8 = e4m3_decode(e4m3_encode((E * p_scale).astype(np.float32)))
+                O[b, h] = (P8 @ ops["vd"][b, hk]) / (p_scale * ls[:, None])
+            else:
+                O[b, h] = (E @ v_exact[b, hk]) / ls[:, None]
+            with np.errstate(divide="ignore"):
+                L[b, h] = np.where(empty, -np.inf, m + np.log(ls) + scale * ops["qk"][b, h, idx])
+            O[b, h][empty] = 0.0
     return O, L
 
 
-def fp8qk_attention_fp64(q_bits, k_bits, v_bits, causal: bool, scale: float, rows=None):
+def sage8_attention_fp64(q_bits, k_bits, v_bits, causal: bool, scale: float, rows=None,
+                         p_scale: float = E4M3_MAX):
+    """Quantised attention with every quantised operand taken from the steps
+    above and every other operation in float64; P is encoded as
+    e4m3(p * p_scale) relative to the exact row maximum (p_scale = 448: the
+    largest weight encodes to the e4m3 maximum). Returns (O, LSE) float64 like
+    ``attention_fp64`` (causal mask bottom-right aligned; a row that sees no
+    key gets O = 0, LSE = -inf).
+
+    This is the 8-bit method's own result without online rescaling; the GPU's
+    8-bit path encodes P relative to a running (lagging) maximum, so the two
+    agree only within the quantisation error, not bit for bit.
+    """
+    ops = quantised_operands(q_bits, k_bits, v_bits, "int8")
+    return _one_shot(ops, None, causal, scale, rows, True, p_scale)
+
+
+def fp8qk_attention_fp64(q_bits, k_bits, v_bits, causal: bool, scale: float, rows=None,
+                         p_scale: float = E4M3_MAX):
     """The FP8-Q K^T variant as a one-shot computation: e4m3 Q and K with one
     scale per 128-token block and no smoothing, P and V as in
     ``sage8_attention_fp64`` (P encoded relative to the exact row maximum)."""
-    B, Hq, Nq, d = q_bits.shape
-    Hkv, Nkv = k_bits.shape[1], k_bits.shape[2]
-    q8, sq = quant_e4m3_blocks(widen_bf16(q_bits).astype(np.float32))
-    k8, sk = quant_e4m3_blocks(widen_bf16(k_bits).astype(np.float32))
-    v8, sv = quant_v_fp8(v_bits)
-    R = Nq if rows is None else rows.shape[-1]
-    O = np.empty((B, Hq, R, d))
-    L = np.empty((B, Hq, R))
-    for b in range(B):
-        for h in range(Hq):
-            hk = _kv_head(h, Hq, Hkv)
-            idx = np.arange(Nq) if rows is None else rows[b, h]
-            qi = e4m3_decode(q8[b, h, idx]) * sq[b, h, idx // BLOCK][:, None].astype(np.float64)
-            kj = e4m3_decode(k8[b, hk]) * sk[b, hk, np.arange(Nkv) // BLOCK][:, None].astype(np.float64)
-            S = scale * (qi @ kj.T)
-            if causal:
-                S = np.where(np.arange(Nkv)[None, :] <= idx[:, None] + (Nkv - Nq), S, -np.inf)
-            m = S.max(axis=1)
-            E = np.exp(S - m[:, None])
-            l = E.sum(axis=1)
-            P8 = e4m3_decode(e4m3_encode((E * E4M3_MAX).astype(np.float32)))
-            Vd = e4m3_decode(v8[b, hk]) * sv[b, hk][None, :].astype(np.float64)
-            O[b, h] = (P8 @ Vd) / (E4M3_MAX * l[:, None])
-            L[b, h] = m + np.log(l)
-    return O, L
+    ops = quantised_operands(q_bits, k_bits, v_bits, "fp8")
+    return _one_shot(ops, None, causal, scale, rows, True, p_scale)
+
+
+def quantised_scores_attention_fp64(q_bits, k_bits, v_bits, causal: bool, scale: float,
+                                    qk_format: str = "int8", rows=None):
+    """The exact softmax of an 8-bit method's dequantised scores, applied to the
+    exact V: everything of the method except the e4m3 rounding of P and V.
+
+    Returns (O_q, LSE_q, A) float64, where A = sum_j P_q[i, j] |V[j, c]| (the
+    P_q-weighted magnitudes that bound the effect of rounding P and V
+    elementwise). Used to split an 8-bit result's error into the part the
+    scores carry (computed here exactly) and the part P and V rounding adds
+    (bounded elementwise).
+    """
+    ops = quantised_operands(q_bits, k_bits, v_bits, qk_format)
+    vx = widen_bf16(v_bits)
+    O, L = _one_shot(ops, vx, causal, scale, rows, False, E4M3_MAX)
+    A, _ = _one_shot(ops, np.abs(vx), causal, scale, rows, False, E4M3_MAX)
+    return O, L, A

@@ -1,6 +1,5 @@
-"""The FMA-pipe exp2 available to the kernels for part of the softmax
-exponentials (the 8-bit kernel's ATTN_Q8_EMU build option, off by default
-because it measured slower on the B200).
+"""The FMA-pipe exp2 the 8-bit kernel uses for 3/8 of its softmax
+exponentials (the rest run on ex2.approx).
 
 Checks that the coefficients in the kernel source are the ones the committed
 fitting script produces (Remez exchange on the relative error of 2^f over

@@ -153,3 +153,262 @@ def test_smoothing_beats_unsmoothed_fp8_on_outlier_channels():
     cos = lambda a: (O * a).sum() / math.sqrt((O * O).sum() * (a * a).sum())  # noqa: E731
     assert cos(Os) >= 0.999 > cos(Of)
     assert np.abs(L - Ls).max() * 5 < np.abs(L - Lf).max()
+
+
+# ---------------------------------------------------------------------------
+# Brute force: the two one-shot 8-bit oracles written out element by element
+# in pure Python (math.fsum, Python's round-half-even, numpy float32 scalars
+# only where the method fixes fp32 division, torch's float8_e4m3fn cast as an
+# e4m3 encoder that shares nothing with oracle.quant8).
+# ---------------------------------------------------------------------------
+def _e4m3_torch(x: float) -> float:
+    """Round to e4m3fn (nearest even) with saturation, through torch's cast."""
+    x = max(-448.0, min(448.0, float(x)))
+    return float(torch.tensor(x, dtype=torch.float32).to(torch.float8_e4m3fn).to(torch.float64))
+
+
+def _blocks(n):
+    return [list(range(s, min(s + 128, n))) for s in range(0, n, 128)]
+
+
+def _quant_rows(rows, fmt):
+    """rows: list of lists of float32 values (one 128-token block per call).
+    Returns (dequantised values as floats, scale)."""
+    amax = max(abs(float(x)) for r in rows for x in r)
+    top = 127.0 if fmt == "int8" else 448.0
+    s = np.float32(np.float32(amax) / np.float32(top)) if amax > 0 else np.float32(1.0)
+    out = []
+    for r in rows:
+        y = [float(np.float32(x) / s) for x in r]
+        if fmt == "int8":
+            out.append([max(-127, min(127, round(v))) * float(s) for v in y])
+        else:
+            out.append([_e4m3_torch(v) * float(s) for v in y])
+    return out, float(s)
+
+
+def _brute_8bit(qb, kb, vb, causal, scale, fmt, p_scale=448.0):
+    """Returns (O, LSE) lists indexed [b][h][i][c] / [b][h][i]."""
+    q, k, v = oracle.widen_bf16(qb), oracle.widen_bf16(kb), oracle.widen_bf16(vb)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nkv = k.shape[1], k.shape[2]
+    g = Hq // Hkv
+    O = np.zeros((B, Hq, Nq, d))
+    L = np.zeros((B, Hq, Nq))
+    for b in range(B):
+        kq, vq, kbar = [], [], []
+        for hk in range(Hkv):
+            if fmt == "int8":
+                kb_ = [np.float32(math.fsum(k[b, hk, j, c] for j in range(Nkv)) / Nkv) for c in range(d)]
+                ks = [[np.float32(np.float32(k[b, hk, j, c]) - kb_[c]) for c in range(d)] for j in range(Nkv)]
+            else:
+                kb_ = [np.float32(0.0)] * d
+                ks = [[np.float32(k[b, hk, j, c]) for c in range(d)] for j in range(Nkv)]
+            kd = []
+            for blk in _blocks(Nkv):
+                deq, _ = _quant_rows([ks[j] for j in blk], fmt)
+                kd += deq
+            vd = [[0.0] * d for _ in range(Nkv)]
+            for c in range(d):
+                amax = max(abs(float(v[b, hk, j, c])) for j in range(Nkv))
+                sv = np.float32(np.float32(amax) / np.float32(448.0)) if amax > 0 else np.float32(1.0)
+                for j in range(Nkv):
+                    vd[j][c] = _e4m3_torch(float(np.float32(v[b, hk, j, c]) / sv)) * float(sv)
+            kq.append(kd)
+            vq.append(vd)
+            kbar.append([float(x) for x in kb_])
+        for h in range(Hq):
+            hk = h // g
+            qd = []
+            for blk in _blocks(Nq):
+                deq, _ = _quant_rows([[np.float32(q[b, h, i, c]) for c in range(d)] for i in blk], fmt)
+                qd += deq
+            for i in range(Nq):
+                vis = [j for j in range(Nkv) if not causal or j <= i + (Nkv - Nq)]
+                if not vis:
+                    L[b, h, i] = -math.inf
+                    continue
+                S = {j: scale * math.fsum(qd[i][c] * kq[hk][j][c] for c in range(d)) for j in vis}
+                m = max(S.values())
+                E = {j: math.exp(S[j] - m) for j in vis}
+                lsum = math.fsum(E.values())
+                P8 = {j: _e4m3_torch(float(np.float32(E[j] * p_scale))) for j in vis}
+                for c in range(d):
+                    O[b, h, i, c] = math.fsum(P8[j] * vq[hk][j][c] for j in vis) / (p_scale * lsum)
+                corr = scale * math.fsum(float(q[b, h, i, c]) * kbar[hk][c] for c in range(d))
+                L[b, h, i] = m + math.log(lsum) + corr
+    return O, L
+
+
+def _tiered_inputs(B, Hq, Hkv, Nq, Nkv, d, seed, dist="normal"):
+    """Seeded inputs whose 128-token blocks differ in magnitude (x1, x8, x1/4,
+    ...), so that per-block scales matter."""
+    q, k, v = make_qkv(B, Hq, Hkv, Nq, Nkv, d, seed=seed, dist=dist)
+    tiers = torch.tensor([1.0, 8.0, 0.25, 3.0])
+    fq = tiers[(torch.arange(Nq) // 128) % 4].view(1, 1, Nq, 1)
+    fk = tiers[(torch.arange(Nkv) // 128 + 1) % 4].view(1, 1, Nkv, 1)
+    return (bf16_bits((q.float() * fq).to(torch.bfloat16)), bf16_bits((k.float() * fk).to(torch.bfloat16)),
+            bf16_bits(v))
+
+
+_BRUTE_CASES = [
+    # B, Hq, Hkv, Nq, Nkv, d, causal
+    (1, 2, 1, 200, 200, 8, False),
+    (1, 2, 1, 200, 200, 8, True),
+    (1, 2, 2, 130, 260, 8, True),    # bottom-right causal, Nq < Nkv
+    (1, 1, 1, 260, 140, 8, True),    # Nq > Nkv: the first rows see no key
+]
+
+
+@pytest.mark.parametrize("fmt", ["int8", "fp8"])
+@pytest.mark.parametrize("case", _BRUTE_CASES)
+def test_one_shot_8bit_matches_brute_force(fmt, case):
+    B, Hq, Hkv, Nq, Nkv, d, causal = case
+    qb, kb, vb = _tiered_inputs(B, Hq, Hkv, Nq, Nkv, d, seed=31 + Nq, dist="outlier_k")
+    sc = 0.3
+    fn = q8.sage8_attention_fp64 if fmt == "int8" else q8.fp8qk_attention_fp64
+    O, L = fn(qb, kb, vb, causal, sc)
+    Ob, Lb = _brute_8bit(qb, kb, vb, causal, sc, fmt)
+    assert np.allclose(O, Ob, rtol=1e-12, atol=1e-12), np.abs(O - Ob).max()
+    fin = np.isfinite(Lb)
+    assert np.array_equal(fin, np.isfinite(L))
+    assert np.allclose(L[fin], Lb[fin], rtol=1e-12, atol=1e-12)
+    if Nq > Nkv and causal:
+        assert np.all(O[:, :, :Nq - Nkv] == 0.0) and np.all(np.isneginf(L[:, :, :Nq - Nkv]))
+
+
+def test_one_shot_8bit_p_scale_matches_brute_force():
+    # P encoded relative to a smaller top code (448 / 16), as the kernel's
+    # lagging reference maximum may leave it
+    qb, kb, vb = _tiered_inputs(1, 2, 1, 200, 200, 8, seed=41, dist="outlier_k")
+    O, L = q8.sage8_attention_fp64(qb, kb, vb, True, 0.3, p_scale=28.0)
+    Ob, Lb = _brute_8bit(qb, kb, vb, True, 0.3, "int8", p_scale=28.0)
+    assert np.allclose(O, Ob, rtol=1e-12, atol=1e-12) and np.allclose(L, Lb, rtol=1e-12, atol=1e-12)
+
+
+def _mutant_fp8(kind):
+    """Planted mistakes in the FP8 Q K^T steps, each a plausible slip."""
+    orig = q8.quant_e4m3_blocks
+    calls = {"n": 0}
+
+    def mutated(x, block=q8.BLOCK):
+        calls["n"] += 1
+        codes, s = orig(x, block)
+        if kind == "global_scale":          # one scale for the whole sequence
+            c1, s1 = orig(x, block=x.shape[2])
+            return c1, np.repeat(s1, s.shape[2], axis=2)
+        if kind == "drop_k_scale" and calls["n"] == 2:   # second call quantises K
+            return codes, np.ones_like(s)
+        if kind == "reversed_blocks":       # scale index transposed within the head
+            return codes, np.ascontiguousarray(s[:, :, ::-1])
+        return codes, s
+    return mutated
+
+
+@pytest.mark.parametrize("kind", ["global_scale", "drop_k_scale", "reversed_blocks"])
+def test_fp8qk_planted_mistakes_fail_the_brute_force(kind, monkeypatch):
+    qb, kb, vb = _tiered_inputs(1, 2, 1, 200, 200, 8, seed=51)
+    Ob, Lb = _brute_8bit(qb, kb, vb, True, 0.3, "fp8")
+    monkeypatch.setattr(q8, "quant_e4m3_blocks", _mutant_fp8(kind))
+    O, L = q8.fp8qk_attention_fp64(qb, kb, vb, True, 0.3)
+    assert max(np.abs(O - Ob).max(), np.abs(L - Lb).max()) > 1e-6
+
+
+@pytest.mark.parametrize("kind", ["no_smoothing", "no_lse_correction", "reversed_blocks"])
+def test_sage8_planted_mistakes_fail_the_brute_force(kind, monkeypatch):
+    qb, kb, vb = _tiered_inputs(1, 2, 1, 200, 200, 8, seed=52, dist="outlier_k")
+    Ob, Lb = _brute_8bit(qb, kb, vb, True, 0.3, "int8")
+    if kind == "no_smoothing":
+        monkeypatch.setattr(q8, "k_channel_mean", lambda kbits: np.zeros(kbits.shape[:2] + kbits.shape[3:], np.float32))
+    elif kind == "no_lse_correction":
+        monkeypatch.setattr(q8, "q_dot_kbar", lambda qbits, kbar, Hkv: np.zeros(qbits.shape[:3]))
+    else:
+        orig = q8.quant_int8_blocks
+        monkeypatch.setattr(q8, "quant_int8_blocks",
+                            lambda x, block=q8.BLOCK: (lambda c, s: (c, np.ascontiguousarray(s[:, :, ::-1])))(*orig(x, block)))
+    O, L = q8.sage8_attention_fp64(qb, kb, vb, True, 0.3)
+    assert max(np.abs(O - Ob).max(), np.abs(L - Lb).max()) > 1e-6
+
+
+def _fp8qk_bound_violations(qb, kb, vb, causal, sc):
+    """Per element: e4m3 rounding of Q and K (relative 2^-4 plus the subnormal
+    quantum 2^-10 of each block scale) moves each score by at most
+    delta_ij = scale * sum_c (|q_ic| e_k + |k_jc| e_q + e_q e_k); P then moves by
+    at most a factor e^{2 Delta_i} (Delta_i = max_j delta_ij), and rounding P
+    (relative 2^-4, absolute 2^-10 / 448 below the normal range) and V
+    (relative 2^-4, absolute 2^-10 * sv) adds the rest; LSE moves by at most
+    Delta_i. Returns the number of outputs of fp8qk_attention_fp64 outside it."""
+    B, Hq, N, d = qb.shape
+    Hkv = kb.shape[1]
+    O, L = oracle.attention_fp64(qb, kb, vb, causal, sc)
+    A, _ = oracle.attention_fp64(qb, kb, vb & np.uint16(0x7FFF), causal, sc)   # sum_j P_ij |v_jc|
+    Of, Lf = q8.fp8qk_attention_fp64(qb, kb, vb, causal, sc)
+    qx, kx, vx = oracle.widen_bf16(qb), oracle.widen_bf16(kb), oracle.widen_bf16(vb)
+    u = 2.0 ** -4 + 2.0 ** -23
+
+    def err(x):   # elementwise e4m3 bound with each 128-token block's own scale
+        e = np.empty_like(x)
+        for s0 in range(0, x.shape[2], 128):
+            blk = x[:, :, s0:s0 + 128]
+            s = np.abs(blk).max(axis=(2, 3), keepdims=True) / 448.0
+            e[:, :, s0:s0 + 128] = u * np.abs(blk) + s * 2.0 ** -10 * (1 + 1e-6)
+        return e
+    eq, ek = err(qx), err(kx)
+    sv = np.abs(vx).max(axis=2) / 448.0 * (1 + 1e-6)
+    vmax = np.abs(vx).max(axis=2)
+    bad = 0
+    for h in range(Hq):
+        hk = h * Hkv // Hq
+        delta = sc * (np.abs(qx[0, h]) @ ek[0, hk].T + eq[0, h] @ np.abs(kx[0, hk]).T + eq[0, h] @ ek[0, hk].T)
+        if causal:
+            delta = np.where(np.arange(N)[None, :] <= np.arange(N)[:, None], delta, 0.0)
+        D = np.exp(2 * delta.max(axis=1))[:, None]
+        n = (np.arange(N) + 1 if causal else np.full(N, N))[:, None]
+        bound = ((D - 1) * A[0, h] + D * A[0, h] * (2.0 ** -3 + 2.0 ** -8)
+                 + (1 + 2.0 ** -4) * sv[0, hk][None, :] * 2.0 ** -10
+                 + n * 2.0 ** -10 / 448.0 * (vmax[0, hk][None, :] * (1 + 2.0 ** -4) + sv[0, hk][None, :] * 2.0 ** -10)
+                 + 1e-12)
+        bad += int(np.sum(np.abs(Of[0, h] - O[0, h]) > bound))
+        bad += int(np.sum(np.abs(Lf[0, h] - L[0, h]) > delta.max(axis=1) + 1e-12))
+    return bad
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8qk_within_e4m3_error_bound_of_exact(causal, monkeypatch):
+    # plain N(0,1) inputs; the scale is small so that the bound is tight
+    # enough for a planted mistake to break it
+    q, k, v = make_qkv(1, 2, 1, 300, 300, 16, seed=61)
+    qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
+    assert _fp8qk_bound_violations(qb, kb, vb, causal, 0.05) == 0
+    monkeypatch.setattr(q8, "quant_e4m3_blocks", _mutant_fp8("drop_k_scale"))
+    assert _fp8qk_bound_violations(qb, kb, vb, causal, 0.05) > 0
+
+
+def test_quantised_scores_attention_exact_when_quantisation_is_exact():
+    """With Q and K whose 128-token blocks are integers times a power of two
+    reaching +-127 (INT8 codes exact), K of zero mean per channel (smoothing
+    subtracts nothing), the quantised scores are the exact scores and the
+    function reduces to the exact definition; A reduces to attention of |V|."""
+    rng = np.random.default_rng(71)
+    B, Hq, Hkv, N, d = 1, 2, 1, 256, 16
+
+    def ints(n, half=False):
+        x = rng.integers(-127, 128, size=(B, Hq if not half else Hkv, n, d)).astype(np.float32)
+        for s0 in range(0, n, 128):
+            x[:, :, s0, 0] = 127.0          # every block reaches the top code
+        return x
+    qf = ints(N) * np.float32(2.0 ** -6)
+    kh = ints(N // 2, half=True) * np.float32(2.0 ** -5)
+    kf = np.concatenate([kh, -kh], axis=2)  # rows in +- pairs: zero mean, blocks reach 127
+    kf = np.concatenate([kf[:, :, 0::2], kf[:, :, 1::2]], axis=2)
+    vf = rng.normal(size=(B, Hkv, N, d)).astype(np.float32)
+    to_bits = lambda a: bf16_bits(torch.from_numpy(a).to(torch.bfloat16))  # noqa: E731
+    qb, kb, vb = to_bits(qf), to_bits(kf), to_bits(vf)
+    assert np.array_equal(oracle.widen_bf16(qb), qf) and np.array_equal(oracle.widen_bf16(kb), kf)
+    assert np.all(oracle.widen_bf16(kb).sum(axis=2) == 0)
+    for causal in (False, True):
+        Oq, Lq, A = q8.quantised_scores_attention_fp64(qb, kb, vb, causal, 0.2)
+        O, L = oracle.attention_fp64(qb, kb, vb, causal, 0.2)
+        Oa, _ = oracle.attention_fp64(qb, kb, vb & np.uint16(0x7FFF), causal, 0.2)
+        assert np.allclose(Oq, O, rtol=1e-12, atol=1e-12) and np.allclose(Lq, L, rtol=1e-12, atol=1e-12)
+        assert np.allclose(A, Oa, rtol=1e-12, atol=1e-12)
