@@ -65,10 +65,23 @@ __device__ __forceinline__ float div_rn(float x, float s, float r) {
   return fmaf(e, r, q0);
 }
 
-__device__ __forceinline__ int8_t quant_i8(float x, float s, float r) {
-  int c = __float2int_rn(div_rn(x, s, r));  // round half to even
-  c = c > 127 ? 127 : (c < -127 ? -127 : c);
-  return static_cast<int8_t>(c);
+// Low bytes of four words, packed: result byte i = byte 0 of word i.
+__device__ __forceinline__ uint32_t low_bytes4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+  uint32_t a, b, r;
+  asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(a) : "r"(w0), "r"(w1));
+  asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(b) : "r"(w2), "r"(w3));
+  asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// INT8 code of x / s as the low byte of a float: for |y| < 2^22, y + 1.5 * 2^23
+// is rounded to an integer, half to even (the float's unit in the last place is
+// 1 there), and its bits are 0x4B400000 + round(y), whose low byte is the
+// two's-complement code. With s = RN(amax / 127) and |x| <= amax, |x / s| <=
+// 127 (1 + 2^-23) rounds to at most 127 in magnitude, so the clamp to +-127 of
+// the method never changes a code.
+__device__ __forceinline__ uint32_t i8_code_word(float x, float s, float r) {
+  return __float_as_uint(div_rn(x, s, r) + 12582912.0f);
 }
 
 // Block-wide max of non-negative floats (256 threads).
@@ -140,21 +153,39 @@ __global__ void __launch_bounds__(kPrepThreads)
 }
 
 // ----------------------------------------------------------------- prepass 2
-// F8 = true (FP8 Q K^T with block scales, no smoothing): kbar is zero.
+// Grid (B * Hkv, D / 32), 256 threads: 32 channels x 8 slices; slice u sums the
+// chunk partials u, u + 8, ... of its channel, the 8 slice sums are added in
+// slice order. F8 = true (FP8 Q K^T with block scales, no smoothing): kbar is zero.
+constexpr int kFinalSlices = 8;
 template <int D, bool F8>
-__global__ void q8_kv_final_kernel(const double* __restrict__ ksum_part,
-                                   const float* __restrict__ vmax_part, int Nkv, int nkb,
-                                   float* __restrict__ kbar, float* __restrict__ sv) {
-  const size_t bh = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
-  const int c = threadIdx.x;
+__global__ void __launch_bounds__(32 * kFinalSlices)
+    q8_kv_final_kernel(const double* __restrict__ ksum_part, const float* __restrict__ vmax_part, int Nkv,
+                       int nkb, float* __restrict__ kbar, float* __restrict__ sv) {
+  __shared__ double ss[kFinalSlices][32];
+  __shared__ float sm[kFinalSlices][32];
+  const size_t bh = blockIdx.x;
+  const int c = blockIdx.y * 32 + (threadIdx.x & 31);
+  const int u = threadIdx.x >> 5;
   double acc = 0.0;
   float m = 0.0f;
-  for (int i = 0; i < nkb; ++i) {
+  for (int i = u; i < nkb; i += kFinalSlices) {
     acc += ksum_part[(bh * nkb + i) * D + c];
     m = fmaxf(m, vmax_part[(bh * nkb + i) * D + c]);
   }
-  kbar[bh * D + c] = F8 ? 0.0f : static_cast<float>(acc / static_cast<double>(Nkv));
-  sv[bh * D + c] = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
+  ss[u][threadIdx.x & 31] = acc;
+  sm[u][threadIdx.x & 31] = m;
+  __syncthreads();
+  if (u == 0) {
+    acc = 0.0;
+    m = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kFinalSlices; ++w) {
+      acc += ss[w][threadIdx.x];
+      m = fmaxf(m, sm[w][threadIdx.x]);
+    }
+    kbar[bh * D + c] = F8 ? 0.0f : static_cast<float>(acc / static_cast<double>(Nkv));
+    sv[bh * D + c] = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
+  }
 }
 
 // ----------------------------------------------------------------- prepass 3
@@ -169,17 +200,18 @@ __device__ __forceinline__ uint2 codes8(const float (&x)[8], float s, float r) {
     return make_uint2(pack_e4m3x2(y[0], y[1]) | (pack_e4m3x2(y[2], y[3]) << 16),
                       pack_e4m3x2(y[4], y[5]) | (pack_e4m3x2(y[6], y[7]) << 16));
   }
-  uint32_t lo = 0, hi = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    lo |= (uint32_t)(uint8_t)quant_i8(x[i], s, r) << (8 * i);
-    hi |= (uint32_t)(uint8_t)quant_i8(x[i + 4], s, r) << (8 * i);
-  }
-  return make_uint2(lo, hi);
+  return make_uint2(low_bytes4(i8_code_word(x[0], s, r), i8_code_word(x[1], s, r), i8_code_word(x[2], s, r),
+                               i8_code_word(x[3], s, r)),
+                    low_bytes4(i8_code_word(x[4], s, r), i8_code_word(x[5], s, r), i8_code_word(x[6], s, r),
+                               i8_code_word(x[7], s, r)));
 }
 
+// One CTA per 128-token block: Q blocks (B * Hq * nqb), then K blocks and V
+// blocks (B * Hkv * nkb each). A thread keeps its rows' raw bf16 vectors in
+// registers (all its loads in flight before the first use) and unpacks them
+// where they are used.
 template <int D, bool F8>
-__global__ void __launch_bounds__(kPrepThreads)
+__global__ void __launch_bounds__(kPrepThreads, 4)  // 4 CTAs per SM hide the loads' latency
     q8_quantize_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                        const uint16_t* __restrict__ v, int B, int Hq, int Hkv, int Nq, int Nkv,
                        int nqb, int nkb, const float* __restrict__ kbar,
@@ -192,76 +224,69 @@ __global__ void __launch_bounds__(kPrepThreads)
   __shared__ float red[kPrepThreads / 32];
   const int tid = threadIdx.x, vc = tid % VPR, rs = tid / VPR;
   const long long n_q_tiles = (long long)B * Hq * nqb;
+  const long long n_k_tiles = (long long)B * Hkv * nkb;
   long long tile = blockIdx.x;
-  float x[NP][8];
+  uint4 raw[NP];
   if (tile < n_q_tiles) {
     const int qb = (int)(tile % nqb);
     const long long bh = tile / nqb;  // b * Hq + h
     const int b = (int)(bh / Hq), h = (int)(bh % Hq);
     const size_t bhk = (size_t)b * Hkv + h / (Hq / Hkv);
-    float amax = 0.0f;
 #pragma unroll
     for (int pp = 0; pp < NP; ++pp) {
       const int t = qb * kTok + rs + pp * RPP;
-      if (t < Nq) {
-        unpack8(*reinterpret_cast<const uint4*>(q + ((size_t)bh * Nq + t) * D + vc * 8), x[pp]);
-      } else {
+      raw[pp] = t < Nq ? *reinterpret_cast<const uint4*>(q + ((size_t)bh * Nq + t) * D + vc * 8)
+                       : make_uint4(0, 0, 0, 0);
+    }
+    float kb[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) x[pp][i] = 0.0f;
-      }
+    for (int i = 0; i < 8; ++i) kb[i] = kbar[bhk * D + vc * 8 + i];
+    float amax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[pp][i]));
+    for (int pp = 0; pp < NP; ++pp) {
+      float x[8];
+      unpack8(raw[pp], x);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
     }
     amax = block_max256(amax, red);
     const float s = amax > 0.0f ? __fdiv_rn(amax, F8 ? 448.0f : 127.0f) : 1.0f;
     const float r_q = __frcp_rn(s);
-    float kb[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) kb[i] = kbar[bhk * D + vc * 8 + i];
 #pragma unroll
     for (int pp = 0; pp < NP; ++pp) {
       const int t = qb * kTok + rs + pp * RPP;
+      float x[8];
+      unpack8(raw[pp], x);
       float dot = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) dot = fmaf(x[pp][i], kb[i], dot);
+      for (int i = 0; i < 8; ++i) dot = fmaf(x[i], kb[i], dot);
 #pragma unroll
       for (int o = VPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
       if (t < Nq) {
-        *reinterpret_cast<uint2*>(q8 + ((size_t)bh * Nq + t) * D + vc * 8) = codes8<F8>(x[pp], s, r_q);
+        *reinterpret_cast<uint2*>(q8 + ((size_t)bh * Nq + t) * D + vc * 8) = codes8<F8>(x, s, r_q);
         if (vc == 0) qk[(size_t)bh * Nq + t] = dot;
       }
     }
     if (tid == 0) sq[(size_t)bh * nqb + qb] = s;
-  } else {
+  } else if (tile < n_q_tiles + n_k_tiles) {
     tile -= n_q_tiles;
     const int kb_i = (int)(tile % nkb);
     const size_t bh = (size_t)(tile / nkb);  // b * Hkv + h
-    float kb[8], svc[8], rsv[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      kb[i] = kbar[bh * D + vc * 8 + i];
-      svc[i] = sv[bh * D + vc * 8 + i];
-      rsv[i] = __frcp_rn(svc[i]);
-    }
-    // K and V rows are loaded raw (bf16) before the block-wide maximum, so that
-    // all of this thread's loads are in flight at once; they are unpacked
-    // where they are used
-    uint4 kraw[NP], vraw[NP];
 #pragma unroll
     for (int pp = 0; pp < NP; ++pp) {
       const int t = kb_i * kTok + rs + pp * RPP;
-      kraw[pp] = t < Nkv ? *reinterpret_cast<const uint4*>(k + (bh * Nkv + t) * D + vc * 8)
-                         : make_uint4(0, 0, 0, 0);
-      vraw[pp] = t < Nkv ? *reinterpret_cast<const uint4*>(v + (bh * Nkv + t) * D + vc * 8)
-                         : make_uint4(0, 0, 0, 0);
+      raw[pp] = t < Nkv ? *reinterpret_cast<const uint4*>(k + (bh * Nkv + t) * D + vc * 8) : make_uint4(0, 0, 0, 0);
     }
+    float kb[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) kb[i] = kbar[bh * D + vc * 8 + i];
     float amax = 0.0f;
 #pragma unroll
     for (int pp = 0; pp < NP; ++pp) {
       const int t = kb_i * kTok + rs + pp * RPP;
       if (t < Nkv) {
         float xk[8];
-        unpack8(kraw[pp], xk);
+        unpack8(raw[pp], xk);
 #pragma unroll
         for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(xk[i] - kb[i]));
       }
@@ -274,13 +299,34 @@ __global__ void __launch_bounds__(kPrepThreads)
       const int t = kb_i * kTok + rs + pp * RPP;
       if (t < Nkv) {
         float xk[8];
-        unpack8(kraw[pp], xk);
+        unpack8(raw[pp], xk);
 #pragma unroll
         for (int i = 0; i < 8; ++i) xk[i] = xk[i] - kb[i];
         *reinterpret_cast<uint2*>(k8 + (bh * Nkv + t) * D + vc * 8) = codes8<F8>(xk, s, r_s);
-        float vf[8];
-        unpack8(vraw[pp], vf);
-        float y[8];
+      }
+    }
+    if (tid == 0) sk[bh * nkb + kb_i] = s;
+  } else {
+    tile -= n_q_tiles + n_k_tiles;
+    const int kb_i = (int)(tile % nkb);
+    const size_t bh = (size_t)(tile / nkb);  // b * Hkv + h
+#pragma unroll
+    for (int pp = 0; pp < NP; ++pp) {
+      const int t = kb_i * kTok + rs + pp * RPP;
+      raw[pp] = t < Nkv ? *reinterpret_cast<const uint4*>(v + (bh * Nkv + t) * D + vc * 8) : make_uint4(0, 0, 0, 0);
+    }
+    float svc[8], rsv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      svc[i] = sv[bh * D + vc * 8 + i];
+      rsv[i] = __frcp_rn(svc[i]);
+    }
+#pragma unroll
+    for (int pp = 0; pp < NP; ++pp) {
+      const int t = kb_i * kTok + rs + pp * RPP;
+      if (t < Nkv) {
+        float vf[8], y[8];
+        unpack8(raw[pp], vf);
 #pragma unroll
         for (int i = 0; i < 8; ++i) y[i] = div_rn(vf[i], svc[i], rsv[i]);
         const uint32_t w0 = pack_e4m3x2(y[0], y[1]) | (pack_e4m3x2(y[2], y[3]) << 16);
@@ -288,7 +334,6 @@ __global__ void __launch_bounds__(kPrepThreads)
         *reinterpret_cast<uint2*>(v8 + (bh * Nkv + t) * D + vc * 8) = make_uint2(w0, w1);
       }
     }
-    if (tid == 0) sk[bh * nkb + kb_i] = s;
   }
 }
 
@@ -721,10 +766,10 @@ cudaError_t launch_q8_d(const Q8Launch& L, cudaStream_t stream) {
   q8_kv_stats_kernel<D><<<g1, kPrepThreads, 0, stream>>>(
       static_cast<const uint16_t*>(L.k), static_cast<const uint16_t*>(L.v), L.p.Nkv, nkb,
       L.ksum_part, L.vmax_part);
-  dim3 g2(L.Hkv, L.B);
-  q8_kv_final_kernel<D, F8><<<g2, D, 0, stream>>>(L.ksum_part, L.vmax_part, L.p.Nkv, nkb, L.kbar,
+  dim3 g2((unsigned)((long long)L.B * L.Hkv), D / 32);
+  q8_kv_final_kernel<D, F8><<<g2, 32 * kFinalSlices, 0, stream>>>(L.ksum_part, L.vmax_part, L.p.Nkv, nkb, L.kbar,
                                               const_cast<float*>(L.p.sv));
-  const long long tiles = (long long)L.B * L.p.Hq * nqb + (long long)L.B * L.Hkv * nkb;
+  const long long tiles = (long long)L.B * L.p.Hq * nqb + 2LL * L.B * L.Hkv * nkb;
   q8_quantize_kernel<D, F8><<<(unsigned)tiles, kPrepThreads, 0, stream>>>(
       static_cast<const uint16_t*>(L.q), static_cast<const uint16_t*>(L.k),
       static_cast<const uint16_t*>(L.v), L.B, L.p.Hq, L.Hkv, L.p.Nq, L.p.Nkv, nqb, nkb, L.kbar,
