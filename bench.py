@@ -170,6 +170,19 @@ def aggregate_tflops(flops_per_rank: float, world: int, max_ms: float) -> float:
     return world * flops_per_rank / (max_ms * 1e-3) / 1e12
 
 
+def workload_config(w: Workload, l2_mode: str) -> dict:
+    """The JSON line's `config`: the same dict for both arms of a workload."""
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nkv": w.Nkv, "d": w.d,
+            "causal": w.causal, "scale": "1/sqrt(d)", "l2": l2_mode,
+            "per_rank": "independent batch (seed + 1000*rank)"}
+
+
+def l2_mode_of(w: Workload) -> str:
+    """Inputs larger than L2, or an L2 flush between steps (as bench_workload)."""
+    in_bytes = 2 * (2 * w.B * w.Hq * w.Nq * w.d + 2 * w.B * w.Hkv * w.Nkv * w.d) + 4 * w.B * w.Hq * w.Nq
+    return "inputs_larger_than_l2" if in_bytes >= 2 * L2_BYTES else "l2_flushed_between_steps"
+
+
 def rank_workload(w: Workload, rank: int) -> Workload:
     """Each rank owns an independent batch of the workload (its own seed)."""
     if rank == 0:
@@ -228,11 +241,10 @@ def bench_workload(w: Workload, steps: int, warmup: int, world: int, rank: int, 
     lse = torch.empty((wr.B, wr.Hq, wr.Nq), dtype=torch.float32, device="cuda")
     in_bytes = 2 * (q.numel() + k.numel() + v.numel()) + 2 * o.numel() + 4 * lse.numel()
     flush = None
-    l2_mode = "inputs_larger_than_l2"
-    if in_bytes < 2 * L2_BYTES:
+    l2_mode = l2_mode_of(w)
+    if l2_mode != "inputs_larger_than_l2":
         scratch = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
         flush = lambda: scratch.zero_()  # noqa: E731
-        l2_mode = "l2_flushed_between_steps"
 
     if w.path == "q8":
         ws = torch.empty(lib_mod.q8_workspace_size(wr.B, wr.Hq, wr.Hkv, wr.Nq, wr.Nkv, wr.d),
@@ -551,9 +563,7 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": "bf16" if w.path != "q8" else "int8 QK^T + e4m3 PV (fp32 accumulation)",
             "data": "synthetic (seeded torch CPU randn -> bf16; outlier-K offsets per head/channel)",
-            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq,
-                       "Nkv": w.Nkv, "d": w.d, "causal": w.causal, "scale": "1/sqrt(d)",
-                       "l2": res["l2"], "per_rank": "independent batch (seed + 1000*rank)"},
+            "config": workload_config(w, res["l2"]),
             "frac_of_bf16_peak": round(value / world / peaks["bf16"], 4),
             "roofline": {"bound": "tensor", "achieved": round(per_launch_tflops, 2),
                          "peak": peaks["bf16"] * (2 if w.path == "q8" else 1), "unit": "TFLOP/s",
@@ -576,6 +586,81 @@ def run_ours(args):
         dist.destroy_process_group()
     if out is not None:
         print(json.dumps(out), flush=True)
+
+
+def kv_shard_inputs(w: Workload, world: int, rank: int):
+    """This rank's inputs for the key-sharded run: every query row and the
+    contiguous key range kv_shard.shard_bounds gives it (CPU bf16 tensors),
+    plus the full key count."""
+    from exact_attention_134_b200.kv_shard import shard_bounds
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.seed, w.dist)
+    lo, hi = shard_bounds(w.Nkv, world, rank)
+    return q, k[:, :, lo:hi].contiguous(), v[:, :, lo:hi].contiguous(), w.Nkv
+
+
+def run_kv_shard(args):
+    """Key-sharded forward of one long-context workload over the ranks (strong
+    scaling: the total work is fixed). Each step runs attn_fwd_partial on the
+    rank's key range, two NCCL all-gathers of the fp32 partials and the merge
+    (kv_shard.attention_kv_sharded); time = max over ranks of the CUDA-event
+    time. One JSON line from rank 0."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import exact_attention_134_b200 as attn
+    from exact_attention_134_b200.kv_shard import attention_kv_sharded
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:  # one rank: a process group of one, so that the same code path runs
+        dist.init_process_group("nccl", store=dist.HashStore(), world_size=1, rank=0)
+    peaks = _peaks()
+    w = WORKLOADS[args.workload]
+    attn.lib()
+    q, ks, vs, n_keys = kv_shard_inputs(w, world, rank)
+    qd, kd, vd = q.cuda(), ks.cuda(), vs.cuda()
+
+    def step():
+        return attention_kv_sharded(qd, kd, vd, n_keys, causal=w.causal)
+
+    clocks = ClockSampler(local)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    times = time_device(step, args.steps, 0)
+    clk = clocks.stop()
+    torch.cuda.synchronize()
+    dist.barrier()
+    st, where = attn.get_status()
+    err = 1.0 if st != 0 else 0.0
+    t = torch.tensor([sum(times), err], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, any_err = float(t[0]), float(t[1])
+    ms = total_ms / args.steps
+    value = w.flops / (ms * 1e-3) / 1e12
+    exchange = world * w.B * w.Hq * w.Nq * (w.d + 1) * 4
+    if rank == 0:
+        out = {"metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+               "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms, 4),
+               "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+               "data": "synthetic (seeded torch CPU randn -> bf16)",
+               "config": {**workload_config(w, "inputs_larger_than_l2"),
+                          "per_rank": "contiguous key range (kv_shard.shard_bounds), all query rows",
+                          "shard": "kv"},
+               "frac_of_bf16_peak": round(value / world / peaks["bf16"], 4),
+               "exchange_bytes_per_rank": exchange,
+               "collectives_per_step": "2 NCCL all-gathers (fp32 O and LSE partials)",
+               "gpu_launches": 2 * args.steps,
+               "clocks": clk, "device_status_error": bool(any_err)}
+        print(json.dumps(out), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
 
 
 def run_bwd_only(args):
@@ -602,31 +687,39 @@ def run_bwd_only(args):
 
 
 def run_reference(args):
-    """The oracle on host cores, timed per step over a bounded sample."""
+    """The oracle, as it stands, on the host cores: each step is a bounded
+    sample of the workload (whole (batch, head) pairs, all query rows), timed
+    by wall clock; `ms_per_step` is that measured time and `value` the sample's
+    FLOPs over it. Under torchrun only rank 0 runs."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     w = WORKLOADS[args.workload]
     q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.seed, w.dist)
+    # per step about 120 s / (steps + warmup) of CPU work, 1..8 s
     budget = max(1.0, min(8.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         cpu_baseline(w, q, k, v, budget_s=budget)
-    vals, samples = [], []
+    vals, secs, samples = [], [], []
     for _ in range(args.steps):
+        t0 = time.perf_counter()
         r = cpu_baseline(w, q, k, v, budget_s=budget)
+        secs.append(time.perf_counter() - t0)
         vals.append(r["value"])
         samples.append(r["sample"])
     value = statistics.mean(vals)
+    ms = statistics.mean(secs) * 1e3
+    sample = (f"each step: whole (batch, head) pairs of the workload in order, all {w.Nq} query rows, "
+              f"until {budget:.1f} s of CPU work; last step: {samples[-1]}")
     out = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
-           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-           "ms_per_step": round(w.flops / (value * 1e12) * 1e3, 3),
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic", "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
-                                           "Nq": w.Nq, "Nkv": w.Nkv, "d": w.d, "causal": w.causal},
+           "data": "synthetic (seeded torch CPU randn -> bf16; outlier-K offsets per head/channel)",
+           "config": workload_config(w, l2_mode_of(w)),
+           "sample": sample,
            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
-                            "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
-                            "sample": samples[-1]},
+                            "cores": len(os.sched_getaffinity(0)), "kind": "oracle", "sample": sample},
            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -645,9 +738,16 @@ def main():
                     help="only the device-timed leg (for profiling runs): no e2e, CPU or extra legs")
     ap.add_argument("--direction", default="fwd", choices=["fwd", "bwd"],
                     help="bwd: time only the backward of --workload (one JSON line)")
+    ap.add_argument("--shard", default="batch", choices=["batch", "kv"],
+                    help="kv: split the keys of --workload over the ranks (key-sharded forward, "
+                         "partial -> NCCL all-gather -> merge; default workload kvcache_128k_q128)")
     args = ap.parse_args()
+    if args.shard == "kv" and args.workload == HEADLINE:
+        args.workload = "kvcache_128k_q128"
     if args.impl == "reference":
         run_reference(args)
+    elif args.shard == "kv":
+        run_kv_shard(args)
     elif args.direction == "bwd":
         run_bwd_only(args)
     else:

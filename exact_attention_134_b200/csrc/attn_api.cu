@@ -87,7 +87,7 @@ attn_status_t check_args(const void* q, const void* k, const void* v, const void
 // 128-byte swizzle (the layout the tcgen05 descriptors expect).
 // (d = 96: 32-column boxes with the 64-byte swizzle, three per 96-column row.)
 // (d = 256 K/V: 64-row boxes, the d = 256 kernel's 64-key tiles.)
-bool make_map(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
+bool encode_map(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * (cuuint64_t)d * 2};
   cuuint32_t box[3] = {d == 96 ? 32u : 64u, d == 256 ? 64u : 128u, 1};
@@ -101,7 +101,7 @@ bool make_map(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
 
 // Packed bf16 tensor [total, H, d] as {d, H, total}; box = 64 columns x 1 head x
 // 128 rows (the same shared-memory layout as the dense box).
-bool make_map_packed(CUtensorMap* m, const void* ptr, int d, int H, int total) {
+bool encode_map_packed(CUtensorMap* m, const void* ptr, int d, int H, int total) {
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)total};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * (cuuint64_t)d * 2};
   cuuint32_t box[3] = {d == 96 ? 32u : 64u, 1, 128};
@@ -114,7 +114,7 @@ bool make_map_packed(CUtensorMap* m, const void* ptr, int d, int H, int total) {
 }
 
 // 8-bit tensor [BH, N, d] as {d, N, BH}; box = d bytes x 128 rows, swizzle = d bytes.
-bool make_map_u8(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
+bool encode_map_u8(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)N * (cuuint64_t)d};
   cuuint32_t box[3] = {(cuuint32_t)d, 128, 1};
@@ -124,6 +124,50 @@ bool make_map_u8(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
                         d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+
+// Encoded tensor maps, cached per calling thread: a map depends only on the
+// pointer, the shape and the layout kind, so a hit returns exactly what the
+// encoder would. Direct-mapped, kMapCacheSlots entries per thread.
+constexpr int kMapCacheSlots = 64;
+struct MapCacheEntry {
+  int kind = -1;  // 0 dense bf16, 1 packed bf16, 2 8-bit
+  const void* ptr = nullptr;
+  long long a = 0, b = 0, c = 0;
+  alignas(64) CUtensorMap map;
+};
+thread_local MapCacheEntry g_map_cache[kMapCacheSlots];
+
+template <typename Encode>
+bool cached_map(CUtensorMap* m, int kind, const void* ptr, long long a, long long b, long long c,
+                Encode encode) {
+  uint64_t h = reinterpret_cast<uintptr_t>(ptr) ^ (uint64_t)kind * 0x9E3779B97F4A7C15ull;
+  h = (h ^ (uint64_t)a * 0xBF58476D1CE4E5B9ull) ^ ((uint64_t)b * 0x94D049BB133111EBull) ^ (uint64_t)c;
+  h ^= h >> 31;
+  MapCacheEntry& e = g_map_cache[h % kMapCacheSlots];
+  if (e.kind == kind && e.ptr == ptr && e.a == a && e.b == b && e.c == c) {
+    *m = e.map;
+    return true;
+  }
+  if (!encode(m)) return false;
+  e.kind = kind;
+  e.ptr = ptr;
+  e.a = a;
+  e.b = b;
+  e.c = c;
+  e.map = *m;
+  return true;
+}
+
+bool make_map(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
+  return cached_map(m, 0, ptr, d, N, BH, [&](CUtensorMap* x) { return encode_map(x, ptr, d, N, BH); });
+}
+bool make_map_packed(CUtensorMap* m, const void* ptr, int d, int H, int total) {
+  return cached_map(m, 1, ptr, d, H, total, [&](CUtensorMap* x) { return encode_map_packed(x, ptr, d, H, total); });
+}
+bool make_map_u8(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
+  return cached_map(m, 2, ptr, d, N, BH, [&](CUtensorMap* x) { return encode_map_u8(x, ptr, d, N, BH); });
 }
 
 // Key-range partial results (dense bf16 kernel only): o_part != null makes the

@@ -721,8 +721,7 @@ cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
   attn_bwd_pre_kernel<D, VL><<<rows_grid, 256, 0, stream>>>(L.pre);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_bwd_main_kernel<D, VL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           BwdCfg<D>::kSmemBytes);
+  e = max_dynamic_smem_once<attn_bwd_main_kernel<D, VL>>(BwdCfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((L.max_kv + kBK - 1) / kBK, L.main.Hkv, L.B);
   attn_bwd_main_kernel<D, VL><<<grid, kThreads, BwdCfg<D>::kSmemBytes, stream>>>(L.tq, L.tk, L.tv, L.tdo,

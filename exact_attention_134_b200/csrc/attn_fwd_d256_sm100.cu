@@ -368,8 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_fwd_d256(const CUtensorMap& tk, const CUtensorMap& tv, const void* q,
                             const FwdParams& p, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_d256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kSmemBytes);
+  cudaError_t e = max_dynamic_smem_once<attn_fwd_d256_kernel>(kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((p.Nq + kBM - 1) / kBM, p.Hq, p.B);
   attn_fwd_d256_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tk, tv, q, p);

@@ -557,8 +557,7 @@ static int smem_bytes() { return FwdCfg<D>::kSmemBytes; }
 template <int D, bool VL, bool PART = false, bool PAIR = false>
 static cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& to, const FwdParams& p, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_bf16_kernel<D, VL, PART, PAIR>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<D>());
+  cudaError_t e = max_dynamic_smem_once<attn_fwd_bf16_kernel<D, VL, PART, PAIR>>(smem_bytes<D>());
   if (e != cudaSuccess) return e;
   // varlen: B = number of sequences; head pairs: Hq / 2 units of 128 rows
   dim3 grid(p.num_row_blocks, PAIR ? p.Hq / 2 : p.Hq, p.B * p.num_splits);

@@ -6,9 +6,27 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/attn.h"
 
 namespace attn_sm100 {
+
+// Raises Kernel's dynamic shared-memory limit to `bytes` once per device: the
+// first launch on a device (with that device current) sets the attribute,
+// later launches skip the runtime call. Devices beyond 64 set it every time.
+template <auto Kernel>
+cudaError_t max_dynamic_smem_once(int bytes) {
+  static std::atomic<unsigned long long> done{0};  // bit d: set on device d
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? 1ull << dev : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // Kernel parameters of the bf16 forward (tensor maps are passed separately).
 struct FwdParams {

@@ -777,8 +777,7 @@ cudaError_t launch_q8_d(const Q8Launch& L, cudaStream_t stream) {
       const_cast<float*>(L.p.qk));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || L.prepass_only) return e;
-  e = cudaFuncSetAttribute(attn_fwd_q8_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Q8Cfg<D>::kSmemBytes);
+  e = max_dynamic_smem_once<attn_fwd_q8_kernel<D, F8>>(Q8Cfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(L.p.num_row_blocks, L.p.Hq, L.B);
   attn_fwd_q8_kernel<D, F8><<<grid, kQ8Threads, Q8Cfg<D>::kSmemBytes, stream>>>(L.tq, L.tk, L.tv, L.to, L.p);

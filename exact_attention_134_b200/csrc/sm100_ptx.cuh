@@ -62,22 +62,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-#ifndef ATTN_TRYWAIT_HINT_NS
-#define ATTN_TRYWAIT_HINT_NS 0
-#endif
-// As mbar_try_wait, with a suspend-time hint (ns) for the waiting thread.
-__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-
 // Bounded wait on phase `parity` of an mbarrier. Returns false when the
 // budget ran out or another role already flagged an abort; the caller then
 // leaves its loop. `abort_flag` lives in shared memory.
@@ -87,9 +71,7 @@ __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity,
   const uint64_t t0 = global_timer_ns();
   // Iteration cap as a second bound in case the timer misbehaves.
   for (uint32_t it = 1; it < (1u << 27); ++it) {
-    if (ATTN_TRYWAIT_HINT_NS > 0 ? mbar_try_wait_hint(bar, parity, ATTN_TRYWAIT_HINT_NS)
-                                 : mbar_try_wait(bar, parity))
-      return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if ((it & 15u) == 0) {
       if (*abort_flag) return false;
       if (global_timer_ns() - t0 > budget_ns) return false;

@@ -61,6 +61,20 @@ def _check(B, Hq, Hkv, Nq, Nkv, d, causal, seed, dist="normal", n_rows=None):
     return mx, mean, dl
 
 
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["outlier_8k_causal", "outlier_8k_full"])
+def test_large_workloads_every_row(name):
+    """Every row of every (batch, head) of the 8k outlier workloads against the
+    fp64 oracle (one (batch, head) per worker process)."""
+    from tests.oracle_pool import attention_fp64_parallel
+    w = WORKLOADS[name]
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.seed, w.dist)
+    o, lse = _run(q, k, v, w.causal)
+    O, L = attention_fp64_parallel(bf16_bits(q), bf16_bits(k), bf16_bits(v), w.causal, w.scale)
+    mx, mean, dl = _compare(o, lse, O, L)
+    assert mx <= MAX_TOL and mean <= MEAN_TOL and dl <= LSE_TOL, (mx, mean, dl)
+
+
 SMALL = [
     # B, Hq, Hkv, Nq, Nkv, d, causal
     (1, 2, 2, 256, 256, 64, False),

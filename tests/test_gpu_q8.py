@@ -99,12 +99,13 @@ def test_prepass_bit_exact_8k_outlier_workload():
     _check_prepass(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.seed, w.dist)
 
 
-def pv_rounding_bound(qb, kb, vb, causal, scale, rows, qk_format, O):
+def pv_rounding_bound(qb, kb, vb, causal, scale, rows, qk_format, O, quantised=None):
     """Per-element bound on |O_gpu - O| for the 8-bit kernel (see the module
-    docstring); O is the exact oracle's output for the same rows."""
+    docstring); O is the exact oracle's output for the same rows, `quantised`
+    the (O_q, LSE_q, A) of quantised_scores_attention_fp64 if already known."""
     B, Hq, Nq, d = qb.shape
     Hkv, Nkv = kb.shape[1], kb.shape[2]
-    Oq, _, A = oq8.quantised_scores_attention_fp64(qb, kb, vb, causal, scale, qk_format, rows=rows)
+    Oq, _, A = quantised or oq8.quantised_scores_attention_fp64(qb, kb, vb, causal, scale, qk_format, rows=rows)
     vx = oracle.widen_bf16(vb)
     sv = (np.abs(vx).max(axis=2) / 448.0 * (1 + 1e-6))[:, np.arange(Hq) // (Hq // Hkv)][:, :, None, :]
     vmax = np.abs(vx).max(axis=2)[:, np.arange(Hq) // (Hq // Hkv)][:, :, None, :]
@@ -115,7 +116,8 @@ def pv_rounding_bound(qb, kb, vb, causal, scale, rows, qk_format, O):
     return core + 2.0 ** -8 * (np.abs(O) + core) + 1e-6
 
 
-def _check_fwd(B, Hq, Hkv, Nq, Nkv, d, causal, seed, dist="normal", n_rows=None, qk_format="int8"):
+def _check_fwd(B, Hq, Hkv, Nq, Nkv, d, causal, seed, dist="normal", n_rows=None, qk_format="int8",
+               parallel=False):
     q, k, v = make_qkv(B, Hq, Hkv, Nq, Nkv, d, seed, dist)
     scale = 1.0 / math.sqrt(d)
     o, lse = attn.attn_fwd_q8(q.cuda(), k.cuda(), v.cuda(), causal=causal, qk_format=qk_format)
@@ -125,7 +127,13 @@ def _check_fwd(B, Hq, Hkv, Nq, Nkv, d, causal, seed, dist="normal", n_rows=None,
     if n_rows:
         rows = sample_rows(Workload("t", B, Hq, Hkv, Nq, Nkv, d, causal, seed), n_rows)
     qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
-    O, L = oracle.attention_fp64(qb, kb, vb, causal, scale, rows=rows)
+    quantised = None
+    if parallel:  # one (batch, head) per worker process
+        from tests.oracle_pool import attention_fp64_parallel, quantised_scores_attention_fp64_parallel
+        O, L = attention_fp64_parallel(qb, kb, vb, causal, scale, rows=rows)
+        quantised = quantised_scores_attention_fp64_parallel(qb, kb, vb, causal, scale, qk_format, rows=rows)
+    else:
+        O, L = oracle.attention_fp64(qb, kb, vb, causal, scale, rows=rows)
     og = o.cpu().float().numpy().astype(np.float64)
     lg = lse.cpu().numpy().astype(np.float64)
     idx = np.arange(Nq)[None, None, :].repeat(B, 0).repeat(Hq, 1) if rows is None else rows
@@ -133,7 +141,7 @@ def _check_fwd(B, Hq, Hkv, Nq, Nkv, d, causal, seed, dist="normal", n_rows=None,
     lg = np.take_along_axis(lg, idx, axis=2)
     assert np.all(np.isfinite(og)) and np.all(np.isfinite(lg))
     err = np.abs(og - O)
-    bound = pv_rounding_bound(qb, kb, vb, causal, scale, rows, qk_format, O)
+    bound = pv_rounding_bound(qb, kb, vb, causal, scale, rows, qk_format, O, quantised)
     assert np.all(err <= bound), (float((err - bound).max()), int((err > bound).sum()))
     if qk_format == "int8":
         cos = float((og * O).sum() / math.sqrt((og * og).sum() * (O * O).sum()))

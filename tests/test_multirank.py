@@ -202,3 +202,64 @@ def test_kv_sharded_rejects_wrong_shards():
         msgs = out[0]
     assert "must hold keys [0, 6) of 6" in msgs[0]
     assert "at least one key" in msgs[1]
+
+
+def _bench_kv_worker(rank, world, port, causal, out):
+    """bench.py --shard kv's host logic on gloo: this rank's shard from
+    bench.kv_shard_inputs, the exchange and merge of kv_shard, oracle partials."""
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    import torch.distributed as dist
+    import bench
+    from exact_attention_134_b200.kv_shard import attention_kv_sharded
+    from synthetic import Workload
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    w = Workload("kv_test", 1, 4, 2, 48, 333, 16, causal, 77)
+    q, ks, vs, n_keys = bench.kv_shard_inputs(w, world, rank)
+    o, lse = attention_kv_sharded(q, ks, vs, n_keys, causal=causal, scale=0.25,
+                                  partial_fn=_oracle_partial, merge_fn=_oracle_merge)
+    shards = [None] * world
+    dist.all_gather_object(shards, ks.float().numpy())
+    out[rank] = (o.numpy(), lse.numpy(), shards)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bench_kv_shard_two_ranks_gloo(causal):
+    """Two gloo ranks run bench.py --shard kv's per-rank inputs through the
+    key-sharded exchange: the shards tile the keys in rank order and every
+    rank's merged result equals the full attention."""
+    import numpy as np
+    import oracle
+    from synthetic import Workload, bf16_bits, make_qkv
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        procs = [ctx.Process(target=_bench_kv_worker, args=(r, world, port, causal, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(180)
+            assert p.exitcode == 0
+        res = dict(out)
+    w = Workload("kv_test", 1, 4, 2, 48, 333, 16, causal, 77)
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.seed, w.dist)
+    full_k = k.float().numpy()
+    assert np.array_equal(np.concatenate(res[0][2], axis=2), full_k)
+    O, L = oracle.attention_fp64(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, 0.25)
+    for r in range(world):
+        o, lse, _ = res[r]
+        assert np.allclose(o, O, rtol=1e-12, atol=1e-12) and np.allclose(lse, L, rtol=1e-12, atol=1e-12)
+
+
+def test_reference_arm_config_is_the_gpu_arms():
+    import bench
+    from synthetic import WORKLOADS
+    for name in ("outlier_8k_causal", "tiny_256_d64"):
+        w = WORKLOADS[name]
+        cfg = bench.workload_config(w, bench.l2_mode_of(w))
+        assert set(cfg) >= {"workload", "scale", "l2", "per_rank"}
+    assert bench.l2_mode_of(WORKLOADS["outlier_8k_causal"]) == "inputs_larger_than_l2"
+    assert bench.l2_mode_of(WORKLOADS["tiny_256_d64"]) == "l2_flushed_between_steps"
