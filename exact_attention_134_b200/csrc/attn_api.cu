@@ -516,6 +516,8 @@ attn_status_t run_bwd(const void* q, const void* k, const void* v, const void* o
 
 namespace attn_sm100 {
 
+attn_status_t cuda_error_status(cudaError_t e) { return cuda_status(e); }
+
 // Internal: the argument checks of attn_fwd / attn_fwd_q8.
 attn_status_t validate_fwd_args(const void* q, const void* k, const void* v, const void* o,
                                 const void* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,

@@ -143,6 +143,10 @@ struct BwdLaunch {
 
 cudaError_t launch_bwd(const BwdLaunch& L, int d, cudaStream_t stream);
 
+// ATTN_OK for cudaSuccess; otherwise remembers `e` for attn_last_cuda_error()
+// (per calling thread) and returns ATTN_ERR_CUDA.
+attn_status_t cuda_error_status(cudaError_t e);
+
 attn_status_t validate_fwd_args(const void* q, const void* k, const void* v, const void* o,
                                 const void* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
                                 int causal, float scale);

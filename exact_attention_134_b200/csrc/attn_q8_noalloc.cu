@@ -12,8 +12,10 @@
 // exits. Host code cannot pass the array's name to a kernel (on the host it is
 // only a stand-in symbol, not a device address), so the first call on each
 // device looks up the array's device address with cudaGetSymbolAddress, with
-// that device current, and caches it; that first call should therefore come
-// before any stream capture.
+// that device current, and caches it. With CUDA's default lazy module loading
+// that lookup is also what loads this file's module onto the device, and so
+// what reserves the 32 MiB: make the first call on each device at start-up,
+// before other allocators take the GPU's memory and before any stream capture.
 #include <mutex>
 
 #include "attn_internal.h"
@@ -61,7 +63,8 @@ attn_status_t attn_fwd_q8_noalloc(const void* q, const void* k, const void* v, v
   if (attn_fwd_q8_workspace_size(B, Hq, Hkv, Nq, Nkv, d) > kAttnQ8StaticScratchBytes)
     return ATTN_ERR_WORKSPACE;
   void* scratch = nullptr;
-  if (scratch_for_current_device(&scratch) != cudaSuccess) return ATTN_ERR_CUDA;
+  const cudaError_t e = scratch_for_current_device(&scratch);
+  if (e != cudaSuccess) return attn_sm100::cuda_error_status(e);
   // Nothing in the scratch has to start at zero: every region the kernels read
   // is written earlier in the same call.
   return attn_sm100::q8_forward_with_workspace(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, causal,

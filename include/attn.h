@@ -247,8 +247,12 @@ ATTN_API attn_status_t attn_fp8_prepass(const void* q, const void* k, const void
  *                  is queued
  *   allocation     none: no cudaMalloc / cudaFree or allocating library call
  *   first call     on each device, looks up the array's device address
- *                  (cudaGetSymbolAddress) with that device current; make the
- *                  first call on a device before any stream capture
+ *                  (cudaGetSymbolAddress) with that device current; with
+ *                  CUDA's default lazy module loading this is also when the
+ *                  32 MiB are reserved on that device, so make the first call
+ *                  at start-up, before other allocators take the GPU's memory
+ *                  and before any stream capture; a failure of the look-up
+ *                  returns ATTN_ERR_CUDA (attn_last_cuda_error has the cause)
  *   concurrency    every call shares the one array: calls whose work overlaps
  *                  on the GPU (different streams, no ordering between them)
  *                  race on it and must be serialised by the caller. The array
