@@ -4,12 +4,18 @@ Prepass: the quantised codes and scales are compared bit for bit with the
 oracle's 8-bit steps (both sides decide every code in fp32 with correctly
 rounded division and round-half-even); q.kbar within fp32 rounding.
 
-Forward: against the EXACT fp64 oracle (not the quantised one) with the 8-bit
-tolerance: cosine >= 0.999 over all compared outputs, max |dO| <= 5e-2 on rows
-that see at least 128 keys (one full K/V tile; rows with fewer keys average too
-few e4m3-rounded terms — the oracle's own one-shot 8-bit result misses 5e-2
-there as well), |dLSE| <= 5e-2, and on EVERY row a per-element bound derived
-from the method's arithmetic (``pv_rounding_bound``):
+Forward: against the EXACT fp64 oracle (not the quantised one):
+  * cosine similarity >= 0.999 over all compared outputs;
+  * |dLSE| <= 5e-2;
+  * max |dO| <= 5e-2 on rows that see at least MANY_KEYS = 512 keys. Rows with
+    fewer keys average too few e4m3-rounded terms for that bound: the 8-bit
+    method itself — the oracle's one-shot quantised attention, exact row
+    maximum, every other operation in fp64 — reaches 0.053 on rows with
+    128-143 keys and 0.047 with 256-383 keys of the 8k outlier workload, and
+    stays at or below 0.028 from 512 keys on (tests/golden/q8_error_by_keys.json,
+    written by tests/golden/q8_error_by_keys.py from the oracle alone);
+  * on EVERY row, every element within a bound derived from the method's
+    arithmetic (``pv_rounding_bound``):
 
     |O_gpu - O| <= |O_q - O| + A (2^-3 + 2^-8 + 2^-10) + sv 2^-10 (1 + 2^-4)
                    + n 2^-10 / 28 (vmax (1 + 2^-4) + sv 2^-10) + bf16 rounding
@@ -37,6 +43,9 @@ from oracle import quant8 as oq8
 from synthetic import WORKLOADS, Workload, bf16_bits, make_qkv, sample_rows
 
 pytestmark = pytest.mark.gpu
+
+# rows with at least this many visible keys are held to max |dO| <= 5e-2 (see above)
+MANY_KEYS = 512
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -146,7 +155,7 @@ def _check_fwd(B, Hq, Hkv, Nq, Nkv, d, causal, seed, dist="normal", n_rows=None,
     if qk_format == "int8":
         cos = float((og * O).sum() / math.sqrt((og * og).sum() * (O * O).sum()))
         nkeys = np.clip(idx + 1 + (Nkv - Nq), 0, Nkv) if causal else np.full_like(idx, Nkv)
-        many = nkeys >= 128
+        many = nkeys >= MANY_KEYS
         assert cos >= 0.999, cos
         if many.any():
             assert err[many].max() <= 5e-2, err[many].max()
@@ -166,6 +175,14 @@ def test_q8_forward_small(shape):
 def test_q8_forward_workloads(name):
     w = WORKLOADS[name]
     _check_fwd(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.causal, w.seed, w.dist, n_rows=w.oracle_rows)
+
+
+@pytest.mark.slow
+def test_q8_forward_every_row_8k_outlier():
+    """Every row of the 8-bit 8k outlier workload against the exact fp64 oracle
+    with the 8-bit tolerance and the per-element bound."""
+    w = WORKLOADS["q8_8k_outlier"]
+    _check_fwd(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.causal, w.seed, w.dist, parallel=True)
 
 
 def test_q8_workspace_errors():
