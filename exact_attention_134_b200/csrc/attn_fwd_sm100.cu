@@ -531,7 +531,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_store_3d(&tm_o, sQ + t * C::kTileBytes + bx * C::kBoxBytes, bx * 64, q0 + t * kTileRowStep,
                          bh_qt);
           tma_store_commit();
-          tma_store_wait_all();
+          // the CTA may exit once the store has read shared memory; its global
+          // writes complete on their own (visible when the kernel ends)
+          tma_store_wait_read();
         } else {
           flag_abort(abort_flag, p.status, 0x400 | t);
         }
