@@ -355,7 +355,7 @@ struct Q8Cfg {
 
 struct Q8Bar {
   static constexpr int kFull = 0, kEmpty = 8, kQFull = 16, kSFull = 17, kPFull = 19,
-                       kOFinal = 21, kEpi = 22, kDrain = 24;
+                       kOFinal = 21, kEpi = 22, kDrain = 24, kSInit = 25;
   static constexpr int kTmemSlotByte = 8 * 32;
   static constexpr int kAbortByte = 8 * 32 + 4;
 };
@@ -367,18 +367,36 @@ __device__ __forceinline__ void q8_flag_abort(volatile int* abort_flag, int* sta
 
 __device__ __forceinline__ bool q8_warp_all(bool v) { return __all_sync(0xffffffffu, v) != 0; }
 
+// Columns of an INT8 score tile that the MMA writes from zero: P (128 e4m3 per
+// row) is stored over them, so they are in use until P.V has read P. The other
+// kTok - kPCols columns are pre-set by the softmax threads to the bits of
+// M = 1.5 * 2^23 and accumulated onto (see the softmax's s32 -> fp32 note).
+constexpr int kPCols = kTok / 4;
+
 // S = Q8 K8^T: INT8 (s32 accumulation) or, with F8, e4m3 (fp32 accumulation).
+// INT8: keys [0, kPCols) into columns [0, kPCols) from zero, keys [kPCols, kTok)
+// accumulated onto the pre-set columns [kPCols, kTok).
 template <int D, bool F8>
 __device__ __forceinline__ void issue_qk_i8(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
-  constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(128, 128) : idesc_s8_s32(128, 128);
+  if constexpr (F8) {
+    constexpr uint32_t idesc = idesc_e4m3_f32(128, 128);
 #pragma unroll
-  for (int kk = 0; kk < D / 32; ++kk) {
-    const uint64_t a = smem_desc_sw(q_smem + kk * 32, 16, 8 * D, D);
-    const uint64_t b = smem_desc_sw(k_smem + kk * 32, 16, 8 * D, D);
-    if (F8)
+    for (int kk = 0; kk < D / 32; ++kk) {
+      const uint64_t a = smem_desc_sw(q_smem + kk * 32, 16, 8 * D, D);
+      const uint64_t b = smem_desc_sw(k_smem + kk * 32, 16, 8 * D, D);
       mma_f8_ss(d_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
-    else
-      mma_i8_ss(d_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+    }
+  } else {
+    constexpr uint32_t idesc_p = idesc_s8_s32(128, kPCols);
+    constexpr uint32_t idesc_rest = idesc_s8_s32(128, kTok - kPCols);
+    // key row r of the tile starts at r * D bytes; kPCols rows are whole swizzle atoms
+    const uint32_t k_rest = k_smem + kPCols * D;
+#pragma unroll
+    for (int kk = 0; kk < D / 32; ++kk) {
+      const uint64_t a = smem_desc_sw(q_smem + kk * 32, 16, 8 * D, D);
+      mma_i8_ss(d_tmem, a, smem_desc_sw(k_smem + kk * 32, 16, 8 * D, D), idesc_p, kk > 0 ? 1u : 0u);
+      mma_i8_ss(d_tmem + kPCols, a, smem_desc_sw(k_rest + kk * 32, 16, 8 * D, D), idesc_rest, 1u);
+    }
   }
 }
 
@@ -447,6 +465,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     }
     mbar_init(bar(Q8Bar::kOFinal), 1);
     mbar_init(bar(Q8Bar::kDrain), 1);
+    mbar_init(bar(Q8Bar::kSInit), 8);  // one arrival per softmax warp
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -507,6 +526,8 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     const uint32_t tO[2] = {tmem + C::kColO0, tmem + C::kColO1};
     const uint32_t q_smem[2] = {sQ, sQ + C::kTileBytes};
     bool ok = q8_warp_all(bounded_wait(bar(Q8Bar::kQFull), 0, abort_flag, budget));
+    // INT8: the softmax threads pre-set the accumulated score columns before S(0)
+    if (!F8 && ok) ok = q8_warp_all(bounded_wait(bar(Q8Bar::kSInit), 0, abort_flag, budget));
     uint32_t slot = 0, v_prev_stage = 0;
     int j = 0;
     for (; j < n_tiles && ok; ++j) {
@@ -598,6 +619,21 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     // only when a tile's maximum exceeds m_ref + kLag
     constexpr float kLag = 4.0f;
 
+    // s32 -> fp32 without a conversion instruction: |s| <= 127 * 127 * d < 2^22,
+    // so the bits of (s + 0x4B400000) are the float M + s exactly, M = 1.5 * 2^23.
+    // The MMA adds s onto columns [kPCols, kTok) pre-set to 0x4B400000 (here for
+    // S(0), after each read of S for the next tile); the columns P is stored over
+    // get the integer add in registers. (The e4m3 MMA accumulates in fp32: no bias.)
+    constexpr uint32_t kMagicBits = 0x4B400000u;
+    if (!F8) {
+#pragma unroll
+      for (int c = kPCols; c < kTok; c += 32) tmem_fill32(tS + c, kMagicBits);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(Q8Bar::kSInit));
+    }
+
     float m_run = -INFINITY;  // reference maximum of scale*log2(e)*S: within kLag below the row maximum
     float l_run = 0.0f;       // sum of 448 * 2^-kLag * 2^(. - m_run)
     bool ok = true;
@@ -617,15 +653,12 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
         tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
       tmem_wait_ld();
       const float f = sq_t * sk_j * p.scale_log2;
-      // s32 -> fp32 without a conversion instruction: |s| <= 127 * 127 * d < 2^22,
-      // so the bits of (s + 0x4B400000) are the float M + s exactly, M = 1.5 * 2^23.
-      // Those floats order like s (same binade), so the row maximum is taken on
-      // them, and M * f is folded into the exponent's bias below. (The e4m3 MMA
-      // already accumulates in fp32: kOff = 0.)
+      // The floats M + s order like s (same binade), so the row maximum is taken
+      // on them, and M * f is folded into the exponent's bias below.
       constexpr float kMagic = 12582912.0f;
       constexpr float kOff = F8 ? 0.0f : kMagic;
 #pragma unroll
-      for (int c = 0; c < (F8 ? 0 : kTok); ++c) sr[c] += 0x4B400000u;
+      for (int c = 0; c < (F8 ? 0 : kPCols); ++c) sr[c] += kMagicBits;
       const int kv0 = j * kTok;
       const bool tile_masked =
           (kv0 + kTok > p.Nkv) || (p.causal && kv0 + kTok - 1 > q0 + t * kTok + diag);
@@ -679,6 +712,12 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
       const float2 acc01 = add2(acc[0], acc[1]), acc23 = add2(acc[2], acc[3]);
       const float row_sum = (acc01.x + acc01.y) + (acc23.x + acc23.y);
       tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&sr[0]));
+      if (!F8) {
+        // S(j) has been read: pre-set the accumulated columns for S(j + 1) (the
+        // MMA writes them only after this step's P-full arrival)
+#pragma unroll
+        for (int c = kPCols; c < kTok; c += 32) tmem_fill32(tS + c, kMagicBits);
+      }
       const bool rescale = (j > 0) && (alpha != 1.0f);
       if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
