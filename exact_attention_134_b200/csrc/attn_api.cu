@@ -62,7 +62,7 @@ int* device_status_ptr() {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // d = 96 is supported by the bf16 kernels only (allow96 = false for the 8-bit
-// paths); d = 256 by the dense bf16 forward only (allow256).
+// paths); d = 256 by the bf16 forward only, dense and packed (allow256).
 attn_status_t check_args(const void* q, const void* k, const void* v, const void* o,
                          const void* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
                          int causal, float scale, bool allow96 = true, bool allow256 = false) {
@@ -100,11 +100,11 @@ bool encode_map(CUtensorMap* m, const void* ptr, int d, int N, long long BH) {
 }
 
 // Packed bf16 tensor [total, H, d] as {d, H, total}; box = 64 columns x 1 head x
-// 128 rows (the same shared-memory layout as the dense box).
+// 128 rows (the same shared-memory layout as the dense box; d = 256: 64 rows).
 bool encode_map_packed(CUtensorMap* m, const void* ptr, int d, int H, int total) {
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)total};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * (cuuint64_t)d * 2};
-  cuuint32_t box[3] = {d == 96 ? 32u : 64u, 1, 128};
+  cuuint32_t box[3] = {d == 96 ? 32u : 64u, 1, d == 256 ? 64u : 128u};
   cuuint32_t elem_strides[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
                         strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -249,7 +249,8 @@ attn_status_t run_fwd_varlen(const void* q, const void* k, const void* v, void* 
   int* status = device_status_ptr();
   if (!status) return ATTN_ERR_CUDA;
   alignas(64) CUtensorMap tq, tk, tv;
-  if (!make_map_packed(&tq, q, d, Hq, total_q) || !make_map_packed(&tk, k, d, Hkv, total_k) ||
+  // d = 256: the d = 256 kernel reads Q rows directly (no Q map)
+  if ((d != 256 && !make_map_packed(&tq, q, d, Hq, total_q)) || !make_map_packed(&tk, k, d, Hkv, total_k) ||
       !make_map_packed(&tv, v, d, Hkv, total_k))
     return ATTN_ERR_CUDA;
   attn_sm100::FwdParams p;
@@ -264,10 +265,11 @@ attn_status_t run_fwd_varlen(const void* q, const void* k, const void* v, void* 
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.causal = causal;
-  const int rows = attn_sm100::fwd_rows_per_cta();
+  const int rows = d == 256 ? attn_sm100::fwd_rows_per_cta_d256() : attn_sm100::fwd_rows_per_cta();
   p.num_row_blocks = (max_seqlen_q + rows - 1) / rows;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
+  if (d == 256) return cuda_status(attn_sm100::launch_fwd_d256(tk, tv, q, p, stream));
   // the output map is unused by the packed path (rows are stored one by one)
   return cuda_status(attn_sm100::launch_fwd_bf16(tq, tk, tv, tq, p, d, stream));
 }
@@ -666,7 +668,8 @@ attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void*
   if (!cu_seqlens_q || !cu_seqlens_k) return ATTN_ERR_INVALID_ARG;
   if (num_seqs <= 0 || max_seqlen_q <= 0) return ATTN_ERR_INVALID_ARG;
   // the dense checks with B = 1 cover pointers, sizes, heads, scale, d and alignment
-  attn_status_t s = check_args(q, k, v, o, lse, 1, Hq, Hkv, total_q, total_k, d, causal, scale);
+  attn_status_t s = check_args(q, k, v, o, lse, 1, Hq, Hkv, total_q, total_k, d, causal, scale,
+                               true, true);
   if (s != ATTN_OK) return s;
   if (num_seqs > 65535) return ATTN_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) | reinterpret_cast<uintptr_t>(cu_seqlens_k)) & 3u)

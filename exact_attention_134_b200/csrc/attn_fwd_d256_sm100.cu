@@ -23,6 +23,10 @@
 // was issued before it (tcgen05 MMAs from one thread execute in order). O is
 // rescaled only when a row's running maximum moves by more than 2^8, and only
 // then does the softmax wait for PV(j-1).
+// VL = true: packed variable-length sequences [total, H, d] (grid z = sequence,
+// rows from cu_seqlens, per-sequence bottom-right causal mask). A K/V tile that
+// runs past its sequence reads the next sequence's rows (or the map's zero
+// fill past the end); those columns are masked to -inf, so P = 0 there.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -90,6 +94,7 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
   }
 }
 
+template <bool VL>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_d256_kernel(const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const void* __restrict__ q,
@@ -105,20 +110,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit: 128 query rows of one (batch, query head)
-  const int nrb = (p.Nq + kBM - 1) / kBM;
-  // causal: row blocks heaviest first across groups of heads (see grouped_heavy_first)
+  // ---- work unit: 128 query rows of one (batch entry or sequence, query head)
+  // dense causal: row blocks heaviest first across groups of heads (see grouped_heavy_first)
   int ux, hq, b;
-  grouped_heavy_first(p.lpt_group, ux, hq, b);
+  grouped_heavy_first(VL ? 0 : p.lpt_group, ux, hq, b);
+  int Lq = p.Nq, Lk = p.Nkv, q_start = 0, k_start = 0;
+  if (VL) {
+    const int sq = blockIdx.z;
+    q_start = min(max(p.cu_q[sq], 0), p.Nq);
+    Lq = min(max(p.cu_q[sq + 1], q_start), p.Nq) - q_start;
+    k_start = min(max(p.cu_k[sq], 0), p.Nkv);
+    Lk = min(max(p.cu_k[sq + 1], k_start), p.Nkv) - k_start;
+    b = 0;
+  }
+  const int nrb = (Lq + kBM - 1) / kBM;
+  if (ux >= nrb) return;  // this sequence has fewer rows (the whole CTA leaves)
   const int row_block = p.causal ? (nrb - 1 - ux) : ux;
   const int hk = hq / (p.Hq / p.Hkv);
   const int q0 = row_block * kBM;
   const int bh_q = b * p.Hq + hq;
   const int bh_kv = b * p.Hkv + hk;
-  const int diag = p.causal ? p.Nkv - p.Nq : 0;  // key j visible to query i iff j <= i + diag
-  int n_tiles = (p.Nkv + kBN - 1) / kBN;
+  const int diag = p.causal ? Lk - Lq : 0;  // key j visible to query i iff j <= i + diag
+  int n_tiles = (Lk + kBN - 1) / kBN;
   if (p.causal) {
-    const int last_key = min(min(q0 + kBM - 1, p.Nq - 1) + diag, p.Nkv - 1);
+    const int last_key = min(min(q0 + kBM - 1, Lq - 1) + diag, Lk - 1);
     n_tiles = last_key < 0 ? 1 : last_key / kBN + 1;
   }
   n_tiles = max(n_tiles, 1);  // a row that sees no key ends with l = 0
@@ -168,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(fb, kTileBytes);
           for (int bx = 0; bx < kBoxes; ++bx)
             tma_load_3d(base + stage * kTileBytes + bx * kBoxBytes, which ? &tm_v : &tm_k, fb, bx * 64,
-                        j * kBN, bh_kv);
+                        VL ? hk : j * kBN, VL ? k_start + j * kBN : bh_kv);
         }
         __syncwarp();
         ++issued;
@@ -231,12 +246,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================================================================ softmax / correction / epilogue
     const int r = threadIdx.x;  // query row within the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(warp << 5) << 16;
-    const int row = q0 + r;
-    const bool row_valid = row < p.Nq;
+    const int row = q0 + r;  // within the sequence
+    const bool row_valid = row < Lq;
+    // element offset of a valid row (row 0 of the unit's sequence otherwise) in Q and O
+    const size_t row_off = VL ? ((size_t)(q_start + (row_valid ? row : 0)) * p.Hq + hq) * kD
+                              : ((size_t)bh_q * p.Nq + (row_valid ? row : 0)) * kD;
     // Q row -> registers -> TMEM (bf16 pairs: column c holds elements 2c, 2c+1)
     {
-      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(q) +
-                                                        ((size_t)bh_q * p.Nq + (row_valid ? row : 0)) * kD);
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(q) + row_off);
 #pragma unroll 1
       for (int c = 0; c < kD / 64; ++c) {
         uint32_t w[32];
@@ -270,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_wait_ld();
       const int kv0 = j * kBN;
-      int lim = p.Nkv - kv0;
+      int lim = Lk - kv0;
       if (p.causal) lim = min(lim, row + diag - kv0 + 1);
       if (lim < kBN) {
 #pragma unroll
@@ -330,8 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue: O / l -> bf16, row stores; LSE
       tc_fence_after();
       const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
-      uint4* const orow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) +
-                                                   ((size_t)bh_q * p.Nq + (row_valid ? row : 0)) * kD);
+      uint4* const orow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + row_off);
 #pragma unroll 1
       for (int c = 0; c < kD / 32; ++c) {
         uint32_t o[32];
@@ -349,7 +365,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (row_valid) p.lse[(size_t)bh_q * p.Nq + row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+      if (row_valid)
+        p.lse[VL ? (size_t)hq * p.Nq + q_start + row : (size_t)bh_q * p.Nq + row] =
+            (m_run + log2f(l_run)) * 0.69314718055994530942f;
     } else if (lane == 0) {
       flag_abort(abort_flag, p.status, 0x300 | (j << 12));
     }
@@ -366,13 +384,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_fwd_d256(const CUtensorMap& tk, const CUtensorMap& tv, const void* q,
-                            const FwdParams& p, cudaStream_t stream) {
-  cudaError_t e = max_dynamic_smem_once<attn_fwd_d256_kernel>(kSmemBytes);
+namespace {
+template <bool VL>
+cudaError_t launch_d256(const CUtensorMap& tk, const CUtensorMap& tv, const void* q,
+                        const FwdParams& p, cudaStream_t stream) {
+  cudaError_t e = max_dynamic_smem_once<attn_fwd_d256_kernel<VL>>(kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.Nq + kBM - 1) / kBM, p.Hq, p.B);
-  attn_fwd_d256_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tk, tv, q, p);
+  // packed: grid x covers the longest sequence (p.num_row_blocks), z = sequence
+  dim3 grid(VL ? p.num_row_blocks : (p.Nq + kBM - 1) / kBM, p.Hq, p.B);
+  attn_fwd_d256_kernel<VL><<<grid, kThreads, kSmemBytes, stream>>>(tk, tv, q, p);
   return cudaGetLastError();
 }
+}  // namespace
+
+cudaError_t launch_fwd_d256(const CUtensorMap& tk, const CUtensorMap& tv, const void* q,
+                            const FwdParams& p, cudaStream_t stream) {
+  return p.cu_q != nullptr ? launch_d256<true>(tk, tv, q, p, stream)
+                           : launch_d256<false>(tk, tv, q, p, stream);
+}
+
+int fwd_rows_per_cta_d256() { return kBM; }
 
 }  // namespace attn_sm100

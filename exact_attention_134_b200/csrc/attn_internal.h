@@ -167,9 +167,10 @@ int fwd_rows_per_cta_paired();
 cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int num_parts,
                          long long rows, int d, void* o, float* lse, cudaStream_t stream);
 
-// Head dim 256 (dense tensors only): K/V tensor maps with 64-row boxes; Q is
-// read directly from global memory.
+// Head dim 256, dense tensors or (p.cu_q set) packed sequences: K/V tensor maps
+// with 64-row boxes; Q is read directly from global memory.
 cudaError_t launch_fwd_d256(const CUtensorMap& tk, const CUtensorMap& tv, const void* q,
                             const FwdParams& p, cudaStream_t stream);
+int fwd_rows_per_cta_d256();
 
 }  // namespace attn_sm100

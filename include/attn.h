@@ -96,6 +96,8 @@ ATTN_API attn_status_t attn_fwd(const void* q, const void* k, const void* v, voi
  *                  offsets outside [0, total] are clamped, never followed)
  *   max_seqlen_q   >= the longest query sequence (sizes the grid; rows beyond
  *                  it are not computed)
+ *   d              64, 96, 128 or 256 (the head dimension up to 256 of the same
+ *                  page's section "FlashAttention-2 (2023)")
  * Allocates nothing; one kernel launch on `stream`.
  */
 ATTN_API attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void* o,

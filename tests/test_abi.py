@@ -107,7 +107,7 @@ def test_varlen_entry_validation(lib):
     assert call(cq=None) == 1 and call(ck=None) == 1
     assert call(n=0) == 1 and call(mq=0) == 1 and call(tq=0) == 1 and call(Hq=3) == 1
     assert call(scale=float("nan")) == 1 and call(causal=3) == 1
-    assert call(d=80) == 2 and call(d=256) == 2 and call(n=70000) == 2
+    assert call(d=80) == 2 and call(d=512) == 2 and call(n=70000) == 2  # d = 256 is supported
     assert call(q=P + 2) == 3 and call(cq=P + 2) == 3
 
 

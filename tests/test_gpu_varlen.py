@@ -85,6 +85,10 @@ VARLEN = [
     ([300, 50, 5], [100, 0, 5], 2, 2, 128, True),            # Lq > Lk, an empty key set
     ([700, 0, 33], [700, 40, 33], 4, 4, 64, True),           # an empty query sequence
     ([129, 64, 300], [129, 500, 300], 4, 2, 96, True),       # head dim 96
+    ([1, 17, 128, 129, 300], None, 4, 2, 256, True),         # head dim 256
+    ([64, 200, 513], [1000, 200, 700], 4, 2, 256, True),     # head dim 256, prefill with a cache
+    ([300, 50, 5], [100, 0, 5], 2, 2, 256, True),            # head dim 256, Lq > Lk, an empty key set
+    ([700, 0, 33], [700, 40, 33], 2, 2, 256, False),         # head dim 256, an empty query sequence
 ]
 
 
@@ -101,8 +105,9 @@ def test_varlen_matches_oracle(case):
     _check(o.cpu().float().numpy(), lse.cpu().numpy(), O, L, packed=True)
 
 
-def test_varlen_equal_lengths_is_bit_identical_to_dense():
-    B, H, N, d = 3, 4, 300, 128
+@pytest.mark.parametrize("d", [128, 256])
+def test_varlen_equal_lengths_is_bit_identical_to_dense(d):
+    B, H, N = 3, 4, 300
     q, k, v = make_qkv(B, H, H, N, N, d, seed=8)
     o_d, l_d = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True)
     pack = lambda x: x.permute(0, 2, 1, 3).reshape(B * N, H, d).contiguous().cuda()  # noqa: E731
@@ -112,9 +117,10 @@ def test_varlen_equal_lengths_is_bit_identical_to_dense():
     assert torch.equal(l_v, l_d.permute(1, 0, 2).reshape(H, B * N))
 
 
-def test_varlen_writes_only_its_rows():
+@pytest.mark.parametrize("d", [64, 256])
+def test_varlen_writes_only_its_rows(d):
     lens = [100, 0, 37]
-    q, k, v, cq, ck = _packed(lens, lens, 2, 2, 64, seed=3)
+    q, k, v, cq, ck = _packed(lens, lens, 2, 2, d, seed=3)
     pad = 4096
     obuf = torch.full((q.numel() + 2 * pad,), 9.0, dtype=torch.bfloat16, device="cuda")
     o = obuf[pad:pad + q.numel()].view(q.shape)
