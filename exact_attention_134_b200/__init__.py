@@ -50,6 +50,7 @@ _SIGNATURES = {
     "attn_fwd_splitkv_num_splits": (_c_int, [_c_int] * 7),
     "attn_fwd_splitkv_workspace_size": (_sz, [_c_int] * 7),
     "attn_fwd_splitkv": (_c_int, [_vp] * 5 + [_c_int] * 7 + [_c_float, _c_int, _vp, _sz, _vp]),
+    "attn_fwd_partial_splitkv": (_c_int, [_vp] * 5 + [_c_int] * 7 + [_c_float, _c_int, _c_int, _vp, _sz, _vp]),
     "attn_fwd_host_buffer_size": (_sz, [_c_int] * 6),
     "attn_fwd_host": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 7 + [_c_float, _vp, _sz, _vp]),
     "attn_fwd_q8_workspace_size": (_sz, [_c_int] * 6),
@@ -148,12 +149,18 @@ def _check_qkv(q, k, v):
 
 
 def attn_fwd_partial(q, k, v, causal: bool = False, scale: float | None = None, kv_tail: int = 0,
-                     out=None, lse=None):
+                     out=None, lse=None, num_splits: int = 0, workspace=None):
     """Attention of all rows of q over the keys of k, v, which are one range of
     a longer key sequence with `kv_tail` more keys after it (the causal mask is
     that sequence's, bottom-right aligned). Returns the range's normalised
     partial result (o fp32 [B, Hq, Nq, d], lse fp32 [B, Hq, Nq]; -inf and
-    O = 0 for a row that sees none of its keys), for merge_partials."""
+    O = 0 for a row that sees none of its keys), for merge_partials.
+
+    num_splits: sub-ranges of the keys run as separate CTAs and merged on the
+    device (attn_fwd_partial_splitkv); <= 0 picks one wave's worth, 1 is the
+    single-launch attn_fwd_partial. workspace: a uint8 CUDA buffer of the
+    library's attn_fwd_splitkv_workspace_size bytes (allocated here if None and
+    needed)."""
     import torch
     B, Hq, Hkv, Nq, Nkv, d = _check_qkv(q, k, v)
     if scale is None:
@@ -162,10 +169,22 @@ def attn_fwd_partial(q, k, v, causal: bool = False, scale: float | None = None, 
         out = torch.empty((B, Hq, Nq, d), dtype=torch.float32, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
-    st = lib().attn_fwd_partial(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                lse.data_ptr(), B, Hq, Hkv, Nq, Nkv, d, int(bool(causal)),
-                                float(scale), int(kv_tail), _stream_handle(q.device))
-    _check(st, "attn_fwd_partial")
+    need = 0 if num_splits == 1 else int(lib().attn_fwd_splitkv_workspace_size(B, Hq, Hkv, Nq, Nkv, d,
+                                                                                 int(num_splits)))
+    if need == 0:
+        st = lib().attn_fwd_partial(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr(), B, Hq, Hkv, Nq, Nkv, d, int(bool(causal)),
+                                    float(scale), int(kv_tail), _stream_handle(q.device))
+        _check(st, "attn_fwd_partial")
+        return out, lse
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = lib().attn_fwd_partial_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                        lse.data_ptr(), B, Hq, Hkv, Nq, Nkv, d, int(bool(causal)),
+                                        float(scale), int(kv_tail), int(num_splits),
+                                        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                        _stream_handle(q.device))
+    _check(st, "attn_fwd_partial_splitkv")
     return out, lse
 
 

@@ -636,6 +636,38 @@ size_t attn_fwd_splitkv_workspace_size(int B, int Hq, int Hkv, int Nq, int Nkv, 
   return plan.splits == 1 ? 0 : splitkv_layout(plan.splits, B, Hq, Nq, d).total;
 }
 
+attn_status_t attn_fwd_partial_splitkv(const void* q, const void* k, const void* v, float* o_part,
+                                       float* lse_part, int B, int Hq, int Hkv, int Nq, int Nkv,
+                                       int d, int causal, float scale, int kv_tail, int num_splits,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  attn_status_t s = check_args(q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nkv, d, causal, scale);
+  if (s != ATTN_OK) return s;
+  if (kv_tail < 0 || (long long)Nkv + kv_tail > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const SplitPlan plan = plan_splits(B, Hq, Hkv, Nq, Nkv, d, num_splits);
+  PartialArgs part;
+  part.kv_tail = kv_tail;
+  if (plan.splits == 1) {  // one range: the partial kernel writes the caller's buffers
+    part.o_part = o_part;
+    return run_fwd(q, k, v, nullptr, lse_part, B, Hq, Hkv, Nq, Nkv, d, causal, scale, st, part);
+  }
+  if ((long long)B * plan.splits > 65535) return ATTN_ERR_UNSUPPORTED;
+  const SplitLayout lay = splitkv_layout(plan.splits, B, Hq, Nq, d);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < lay.total) return ATTN_ERR_WORKSPACE;
+  uint8_t* const ws = static_cast<uint8_t*>(workspace);
+  float* const o_parts = reinterpret_cast<float*>(ws);
+  float* const lse_parts = reinterpret_cast<float*>(ws + lay.lse_off);
+  part.o_part = o_parts;
+  part.num_splits = plan.splits;
+  part.kv_chunk = plan.chunk;
+  s = run_fwd(q, k, v, nullptr, lse_parts, B, Hq, Hkv, Nq, Nkv, d, causal, scale, st, part);
+  if (s != ATTN_OK) return s;
+  // the merged result of the sub-ranges is the partial result of the whole range (fp32)
+  return cuda_status(attn_sm100::launch_merge(o_parts, lse_parts, plan.splits,
+                                              (long long)B * Hq * Nq, d, o_part, lse_part, st,
+                                              true));
+}
+
 attn_status_t attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
                                int B, int Hq, int Hkv, int Nq, int Nkv, int d, int causal,
                                float scale, int num_splits, void* workspace,

@@ -9,8 +9,10 @@
 // exact in real arithmetic. A part with LSE_s = -inf (no visible key) has
 // weight 0; a row with no visible key in any part gets O = 0, LSE = -inf.
 //
-// HBM-bound: reads num_parts * (4 d + 4) bytes per row, writes 2 d + 4.
-// d / 4 threads per row (one float4 of every part each), 8 rows per CTA.
+// HBM-bound: reads num_parts * (4 d + 4) bytes per row, writes 2 d + 4 (bf16 O)
+// or 4 d + 4 (fp32 O: the merged result is itself a partial over the union of
+// the ranges, for a later merge). d / 4 threads per row (one float4 of every
+// part each), 8 rows per CTA.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -28,10 +30,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
   return r;
 }
 
-template <int D>
+template <int D, bool F32>
 __global__ void __launch_bounds__(D / 4 * kRowsPerCta)
     attn_merge_kernel(const float* __restrict__ o_parts, const float* __restrict__ lse_parts,
-                      int num_parts, long long rows, uint16_t* __restrict__ o,
+                      int num_parts, long long rows, void* __restrict__ o,
                       float* __restrict__ lse) {
   constexpr int kT = D / 4;  // threads per row
   const int c4 = threadIdx.x % kT;
@@ -53,32 +55,42 @@ __global__ void __launch_bounds__(D / 4 * kRowsPerCta)
     }
   }
   const float inv = total > 0.0f ? 1.0f / total : 0.0f;
-  uint2 out;
-  out.x = pack_bf16x2_rn(acc.x * inv, acc.y * inv);
-  out.y = pack_bf16x2_rn(acc.z * inv, acc.w * inv);
-  reinterpret_cast<uint2*>(o + r * D)[c4] = out;
+  if (F32) {
+    reinterpret_cast<float4*>(static_cast<float*>(o) + r * D)[c4] =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  } else {
+    uint2 out;
+    out.x = pack_bf16x2_rn(acc.x * inv, acc.y * inv);
+    out.y = pack_bf16x2_rn(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(static_cast<uint16_t*>(o) + r * D)[c4] = out;
+  }
   if (c4 == 0) lse[r] = (m == -INFINITY) ? -INFINITY : m + logf(total);
 }
 
 template <int D>
 cudaError_t launch_merge_d(const float* o_parts, const float* lse_parts, int num_parts,
-                           long long rows, void* o, float* lse, cudaStream_t stream) {
+                           long long rows, void* o, float* lse, bool o_fp32, cudaStream_t stream) {
   const long long blocks = (rows + kRowsPerCta - 1) / kRowsPerCta;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  attn_merge_kernel<D><<<(unsigned)blocks, D / 4 * kRowsPerCta, 0, stream>>>(
-      o_parts, lse_parts, num_parts, rows, static_cast<uint16_t*>(o), lse);
+  if (o_fp32)
+    attn_merge_kernel<D, true><<<(unsigned)blocks, D / 4 * kRowsPerCta, 0, stream>>>(
+        o_parts, lse_parts, num_parts, rows, o, lse);
+  else
+    attn_merge_kernel<D, false><<<(unsigned)blocks, D / 4 * kRowsPerCta, 0, stream>>>(
+        o_parts, lse_parts, num_parts, rows, o, lse);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int num_parts,
-                         long long rows, int d, void* o, float* lse, cudaStream_t stream) {
+                         long long rows, int d, void* o, float* lse, cudaStream_t stream,
+                         bool o_fp32) {
   switch (d) {
-    case 64: return launch_merge_d<64>(o_parts, lse_parts, num_parts, rows, o, lse, stream);
-    case 96: return launch_merge_d<96>(o_parts, lse_parts, num_parts, rows, o, lse, stream);
-    case 128: return launch_merge_d<128>(o_parts, lse_parts, num_parts, rows, o, lse, stream);
-    case 256: return launch_merge_d<256>(o_parts, lse_parts, num_parts, rows, o, lse, stream);
+    case 64: return launch_merge_d<64>(o_parts, lse_parts, num_parts, rows, o, lse, o_fp32, stream);
+    case 96: return launch_merge_d<96>(o_parts, lse_parts, num_parts, rows, o, lse, o_fp32, stream);
+    case 128: return launch_merge_d<128>(o_parts, lse_parts, num_parts, rows, o, lse, o_fp32, stream);
+    case 256: return launch_merge_d<256>(o_parts, lse_parts, num_parts, rows, o, lse, o_fp32, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -3,8 +3,10 @@
 For a context too long for one GPU's share of the work, each rank holds one
 contiguous range of the keys and values and all query rows. Each computes
 its range's partial result with ``attn_fwd_partial`` (normalised O_r in fp32
-and LSE_r), the ranks all-gather the partials (NCCL over NVLink), and every
-rank merges them with ``merge_partials``:
+and LSE_r; when the range's own grid would leave SMs idle, its keys are split
+over more CTAs and merged on the device first), the ranks all-gather the
+partials (NCCL over NVLink), and every rank merges them with
+``merge_partials``:
 
     LSE = ln sum_r exp(LSE_r),   O = sum_r exp(LSE_r - LSE) O_r,
 

@@ -171,6 +171,23 @@ ATTN_API attn_status_t attn_fwd_splitkv(const void* q, const void* k, const void
                                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_fwd_partial_splitkv — attn_fwd_partial (same arguments, mask and
+ * results) with the range's keys split into sub-ranges run as separate CTAs
+ * and merged on the device into the fp32 partial result of the whole range
+ * (the merge above, with fp32 O): for a rank of a key-sharded forward whose
+ * B * Hq * ceil(Nq / 256) CTAs would leave SMs idle. num_splits, workspace and
+ * the failure codes as attn_fwd_splitkv (the same attn_fwd_splitkv_num_splits
+ * and attn_fwd_splitkv_workspace_size apply). One range: one launch, no
+ * workspace; otherwise two launches (partials, merge).
+ */
+ATTN_API attn_status_t attn_fwd_partial_splitkv(const void* q, const void* k, const void* v,
+                                                float* o_part, float* lse_part, int B, int Hq,
+                                                int Hkv, int Nq, int Nkv, int d, int causal,
+                                                float scale, int kv_tail, int num_splits,
+                                                void* workspace, size_t workspace_bytes,
+                                                void* stream);
+
+/*
  * attn_fwd_host — the same operation on HOST buffers, for callers whose data
  * lives in host memory. Copies q, k, v into `dev_buf` (a device buffer of at
  * least attn_fwd_host_buffer_size() bytes, 16-byte aligned, owned by the

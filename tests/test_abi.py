@@ -177,3 +177,10 @@ def test_splitkv_plan_and_validation(lib):
                                     nbytes, None)
     assert call(ws=None) == 6 and call(ws=P + 8) == 6 and call(nbytes=need - 1) == 6
     assert call(d=256) == 2 and call(B=20000, S=64) == 2
+
+    # the split partial of a key range: same plan and workspace, plus kv_tail
+    def pcall(ws=P, nbytes=need, d=128, tail=0, o=P):
+        return lib.attn_fwd_partial_splitkv(P, P, P, o, P, 1, 32, 8, 128, 131072, d, 1, 0.1, tail, 0,
+                                            ws, nbytes, None)
+    assert pcall(ws=None) == 6 and pcall(nbytes=need - 1) == 6
+    assert pcall(tail=-1) == 1 and pcall(o=None) == 1 and pcall(d=256) == 2

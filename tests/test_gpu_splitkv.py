@@ -59,13 +59,17 @@ PARTIAL = [
 ]
 
 
+@pytest.mark.parametrize("num_splits", [1, 3])
 @pytest.mark.parametrize("case", PARTIAL, ids=[str(c) for c in PARTIAL])
-def test_partial_matches_oracle(case):
+def test_partial_matches_oracle(case, num_splits):
+    """num_splits = 1: one launch (attn_fwd_partial); 3: the range's keys in
+    up to three sub-ranges merged on the device (attn_fwd_partial_splitkv)."""
     B, Hq, Hkv, Nq, lo, n, tail, d, causal = case
     q, k, v = make_qkv(B, Hq, Hkv, Nq, lo + n + tail, d, seed=sum(case))
     scale = 1 / math.sqrt(d)
     ks, vs = k[:, :, lo:lo + n].contiguous(), v[:, :, lo:lo + n].contiguous()
-    o, lse = attn.attn_fwd_partial(q.cuda(), ks.cuda(), vs.cuda(), causal=causal, kv_tail=tail)
+    o, lse = attn.attn_fwd_partial(q.cuda(), ks.cuda(), vs.cuda(), causal=causal, kv_tail=tail,
+                                   num_splits=num_splits)
     _status_ok()
     assert o.dtype == torch.float32
     O, L = oracle.attention_partial_fp64(bf16_bits(q), bf16_bits(k), bf16_bits(v), lo, lo + n,
@@ -156,6 +160,31 @@ def test_splitkv_long_cache_sampled_rows():
     _status_ok()
     rows = sample_rows(w, 8)
     O, L = oracle.attention_fp64(bf16_bits(q), bf16_bits(k), bf16_bits(v), False, w.scale, rows=rows)
+    og = np.take_along_axis(o.float().cpu().numpy().astype(np.float64), rows[..., None], axis=2)
+    lg = np.take_along_axis(lse.cpu().numpy().astype(np.float64), rows, axis=2)
+    d = np.abs(og - O)
+    assert d.max() <= MAX_TOL and d.mean() <= MEAN_TOL and np.abs(lg - L).max() <= LSE_TOL
+
+
+def test_partial_split_long_range_sampled_rows():
+    """Two halves of the long-cache shape's keys (causal, the first half with the
+    second as its tail), each an automatically split partial (many sub-ranges
+    merged on the device in fp32), then merged: 8 sampled rows per head
+    against the full oracle."""
+    from synthetic import Workload
+    w = Workload("kvcache_causal", 1, 32, 8, 128, 131072, 128, True, 1011)
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.seed)
+    qc = q.cuda()
+    half = w.Nkv // 2
+    assert attn.splitkv_num_splits(w.B, w.Hq, w.Hkv, w.Nq, half, w.d) > 1
+    parts = [attn.attn_fwd_partial(qc, k[:, :, lo:lo + half].contiguous().cuda(),
+                                   v[:, :, lo:lo + half].contiguous().cuda(), causal=True,
+                                   kv_tail=w.Nkv - lo - half)
+             for lo in (0, half)]
+    o, lse = attn.merge_partials(torch.stack([p[0] for p in parts]), torch.stack([p[1] for p in parts]))
+    _status_ok()
+    rows = sample_rows(w, 8)
+    O, L = oracle.attention_fp64(bf16_bits(q), bf16_bits(k), bf16_bits(v), True, w.scale, rows=rows)
     og = np.take_along_axis(o.float().cpu().numpy().astype(np.float64), rows[..., None], axis=2)
     lg = np.take_along_axis(lse.cpu().numpy().astype(np.float64), rows, axis=2)
     d = np.abs(og - O)
