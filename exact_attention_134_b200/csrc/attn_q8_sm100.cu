@@ -7,7 +7,8 @@
 //
 // Steps (one stream, four launches):
 //   1. kv_stats   per 128-token chunk: fp64 partial sums of K (per channel),
-//                 partial max |V| (per channel)
+//                 partial max |V| (per channel); the FP8 Q K^T variant (no
+//                 smoothing) reads V only
 //   2. kv_final   K channel mean kbar (fp64 sum / Nkv, rounded once to fp32),
 //                 V channel scale sv = max|V| / 448
 //   3. quantize   Q -> INT8, one fp32 scale per 128-token block, plus
@@ -99,7 +100,8 @@ __device__ __forceinline__ float block_max256(float v, float* red) {
 }
 
 // ----------------------------------------------------------------- prepass 1
-template <int D>
+// F8 = true (no smoothing): K is not read; only the V maxima are formed.
+template <int D, bool F8>
 __global__ void __launch_bounds__(kPrepThreads)
     q8_kv_stats_kernel(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, int Nkv,
                        int nkb, double* __restrict__ ksum_part, float* __restrict__ vmax_part) {
@@ -120,7 +122,7 @@ __global__ void __launch_bounds__(kPrepThreads)
   for (int pp = 0; pp < NP; ++pp) {  // issue every load of the chunk before using any
     const int t = t0 + rs + pp * RPP;
     const size_t off = (bh * Nkv + (t < Nkv ? t : 0)) * D + vc * 8;
-    kv[pp] = t < Nkv ? *reinterpret_cast<const uint4*>(k + off) : make_uint4(0, 0, 0, 0);
+    kv[pp] = (!F8 && t < Nkv) ? *reinterpret_cast<const uint4*>(k + off) : make_uint4(0, 0, 0, 0);
     vv[pp] = t < Nkv ? *reinterpret_cast<const uint4*>(v + off) : make_uint4(0, 0, 0, 0);
   }
 #pragma unroll
@@ -130,13 +132,13 @@ __global__ void __launch_bounds__(kPrepThreads)
     unpack8(vv[pp], vf);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      s[i] += static_cast<double>(kf[i]);
+      if (!F8) s[i] += static_cast<double>(kf[i]);
       mx[i] = fmaxf(mx[i], fabsf(vf[i]));
     }
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    ssum[rs][vc * 8 + i] = s[i];
+    if (!F8) ssum[rs][vc * 8 + i] = s[i];
     smax[rs][vc * 8 + i] = mx[i];
   }
   __syncthreads();
@@ -144,10 +146,10 @@ __global__ void __launch_bounds__(kPrepThreads)
     double acc = 0.0;
     float m = 0.0f;
     for (int r = 0; r < RPP; ++r) {
-      acc += ssum[r][tid];
+      if (!F8) acc += ssum[r][tid];
       m = fmaxf(m, smax[r][tid]);
     }
-    ksum_part[(bh * nkb + blockIdx.x) * D + tid] = acc;
+    if (!F8) ksum_part[(bh * nkb + blockIdx.x) * D + tid] = acc;
     vmax_part[(bh * nkb + blockIdx.x) * D + tid] = m;
   }
 }
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(32 * kFinalSlices)
   double acc = 0.0;
   float m = 0.0f;
   for (int i = u; i < nkb; i += kFinalSlices) {
-    acc += ksum_part[(bh * nkb + i) * D + c];
+    if (!F8) acc += ksum_part[(bh * nkb + i) * D + c];  // (F8: not written by the statistics)
     m = fmaxf(m, vmax_part[(bh * nkb + i) * D + c]);
   }
   ss[u][threadIdx.x & 31] = acc;
@@ -802,7 +804,7 @@ template <int D, bool F8>
 cudaError_t launch_q8_d(const Q8Launch& L, cudaStream_t stream) {
   const int nqb = L.p.nqb, nkb = L.p.nkb;
   dim3 g1(nkb, L.Hkv, L.B);
-  q8_kv_stats_kernel<D><<<g1, kPrepThreads, 0, stream>>>(
+  q8_kv_stats_kernel<D, F8><<<g1, kPrepThreads, 0, stream>>>(
       static_cast<const uint16_t*>(L.k), static_cast<const uint16_t*>(L.v), L.p.Nkv, nkb,
       L.ksum_part, L.vmax_part);
   dim3 g2((unsigned)((long long)L.B * L.Hkv), D / 32);
