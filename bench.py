@@ -297,9 +297,11 @@ def bench_workload(w: Workload, steps: int, warmup: int, world: int, rank: int, 
     return res
 
 
-def bench_q8(w: Workload, steps: int, warmup: int, world: int, rank: int, lib_mod):
-    """8-bit path: time of the whole call (3 prepass launches + main kernel) and
-    of the prepass alone; the main kernel's share is the difference."""
+def bench_q8(w: Workload, steps: int, warmup: int, world: int, rank: int, lib_mod,
+             qk_format: str = "int8"):
+    """8-bit path (INT8 Q K^T after smoothing, or with qk_format="fp8" FP8 Q K^T
+    with block scales): time of the whole call (3 prepass launches + main
+    kernel) and of the prepass alone; the main kernel's share is the difference."""
     import torch
     wr = rank_workload(w, rank)
     q, k, v = make_qkv(wr.B, wr.Hq, wr.Hkv, wr.Nq, wr.Nkv, wr.d, wr.seed, wr.dist)
@@ -310,10 +312,11 @@ def bench_q8(w: Workload, steps: int, warmup: int, world: int, rank: int, lib_mo
                      dtype=torch.uint8, device="cuda")
 
     def full():
-        lib_mod.attn_fwd_q8(qd, kd, vd, causal=w.causal, workspace=ws, out=o, lse=lse)
+        lib_mod.attn_fwd_q8(qd, kd, vd, causal=w.causal, workspace=ws, out=o, lse=lse,
+                            qk_format=qk_format)
 
     def pre():
-        lib_mod.q8_prepass(qd, kd, vd, ws)
+        lib_mod.q8_prepass(qd, kd, vd, ws, qk_format=qk_format)
 
     _barrier(world)
     t_full = time_device(full, steps, max(warmup, 3))
@@ -531,17 +534,21 @@ def run_ours(args):
                                                                    attn, peaks["bf16"])
         torch.cuda.empty_cache()
         wq = WORKLOADS["q8_8k_outlier"]
-        full_ms, pre_ms = bench_q8(wq, max(3, args.steps // 2), 3, world, rank, attn)
         fp8_peak = 2.0 * peaks["bf16"]
-        extras["q8_8k_outlier"] = {
-            "tflops": round(world * wq.flops / (full_ms * 1e-3) / 1e12, 1),
-            "ms_per_step": round(full_ms, 4), "prepass_ms": round(pre_ms, 4),
-            "main_ms": round(full_ms - pre_ms, 4),
-            "main_tflops": round(world * wq.flops / ((full_ms - pre_ms) * 1e-3) / 1e12, 1),
-            "frac_of_fp8_peak_main": round(wq.flops / ((full_ms - pre_ms) * 1e-3) / 1e12 / fp8_peak, 4),
-            "fp8_peak": f"{fp8_peak:.0f} TFLOP/s = 2 x measured bf16 (nominal fp8/bf16 ratio)",
-            "l2": "inputs_larger_than_l2"}
-        torch.cuda.empty_cache()
+        # the same workload through both 8-bit variants: INT8 Q K^T after K
+        # smoothing, and FP8 e4m3 Q K^T with block scales (no smoothing)
+        for line, fmt in (("q8_8k_outlier", "int8"), ("fp8qk_8k_outlier", "fp8")):
+            full_ms, pre_ms = bench_q8(wq, max(3, args.steps // 2), 3, world, rank, attn, qk_format=fmt)
+            extras[line] = {
+                "qk_format": fmt,
+                "tflops": round(world * wq.flops / (full_ms * 1e-3) / 1e12, 1),
+                "ms_per_step": round(full_ms, 4), "prepass_ms": round(pre_ms, 4),
+                "main_ms": round(full_ms - pre_ms, 4),
+                "main_tflops": round(world * wq.flops / ((full_ms - pre_ms) * 1e-3) / 1e12, 1),
+                "frac_of_fp8_peak_main": round(wq.flops / ((full_ms - pre_ms) * 1e-3) / 1e12 / fp8_peak, 4),
+                "fp8_peak": f"{fp8_peak:.0f} TFLOP/s = 2 x measured bf16 (nominal fp8/bf16 ratio)",
+                "l2": "inputs_larger_than_l2"}
+            torch.cuda.empty_cache()
     out = None
     if rank == 0:
         cpu = None

@@ -27,6 +27,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "attn_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -37,12 +39,24 @@ namespace {
 constexpr int kQ8Threads = 320;
 // Exponentials of the softmax: of every 8 groups of 4, the first kPolyOf8 are
 // evaluated by exp2_poly2 on the FMA pipe, the rest by ex2.approx. The 8-bit
-// softmax's e4m3 packing competes with ex2 for issue; moving 3/8 of the
-// exponentials off it shortened the loop by ~9 % in a register-only B200
-// measurement of the same instruction mix (1/8 and 1/2 were slower).
-constexpr int kPolyOf8 = 3;
+// softmax's e4m3 packing competes with ex2 for issue, so moving some of the
+// exponentials off it pays. Measured on the B200 (8k causal outlier workload,
+// main kernel): FP8 Q K^T 0.806 / 0.797 / 0.824 / 0.859 / 0.945 ms for 1 / 2 /
+// 3 / 4 / 5 of 8; INT8 0.904 ms for 2 of 8, 0.910 for 3. (The same fraction in
+// runs of 16 groups, e.g. the first 4 of 16, is slower than 2 of every 8.)
+constexpr int kPolyOf8 = 2;
 constexpr int kTok = 128;         // tokens per quantisation block == MMA tile rows
 constexpr int kPrepThreads = 256;
+
+// Programmatic dependent launch: the four launches of a call form a chain in
+// which each may be scheduled while its predecessor's last CTAs still run.
+// A kernel lets its dependent launch once all its CTAs have started, and
+// waits for its predecessor's completion (and memory) before it reads
+// anything the predecessor wrote; both are no-ops without the launch attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -112,6 +126,7 @@ __global__ void __launch_bounds__(kPrepThreads)
   const int tid = threadIdx.x, vc = tid % VPR, rs = tid / VPR;
   const size_t bh = (size_t)blockIdx.z * gridDim.y + blockIdx.y;
   const int t0 = blockIdx.x * kTok;
+  pdl_launch_dependents();
   double s[8];
   float mx[8];
 #pragma unroll
@@ -168,6 +183,8 @@ __global__ void __launch_bounds__(32 * kFinalSlices)
   const size_t bh = blockIdx.x;
   const int c = blockIdx.y * 32 + (threadIdx.x & 31);
   const int u = threadIdx.x >> 5;
+  pdl_launch_dependents();
+  pdl_wait();  // the statistics' partials
   double acc = 0.0;
   float m = 0.0f;
   for (int i = u; i < nkb; i += kFinalSlices) {
@@ -229,6 +246,7 @@ __global__ void __launch_bounds__(kPrepThreads, 4)  // 4 CTAs per SM hide the lo
   const long long n_k_tiles = (long long)B * Hkv * nkb;
   long long tile = blockIdx.x;
   uint4 raw[NP];
+  pdl_launch_dependents();
   if (tile < n_q_tiles) {
     const int qb = (int)(tile % nqb);
     const long long bh = tile / nqb;  // b * Hq + h
@@ -240,6 +258,7 @@ __global__ void __launch_bounds__(kPrepThreads, 4)  // 4 CTAs per SM hide the lo
       raw[pp] = t < Nq ? *reinterpret_cast<const uint4*>(q + ((size_t)bh * Nq + t) * D + vc * 8)
                        : make_uint4(0, 0, 0, 0);
     }
+    pdl_wait();  // kbar (the raw Q loads above are already in flight)
     float kb[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) kb[i] = kbar[bhk * D + vc * 8 + i];
@@ -279,6 +298,7 @@ __global__ void __launch_bounds__(kPrepThreads, 4)  // 4 CTAs per SM hide the lo
       const int t = kb_i * kTok + rs + pp * RPP;
       raw[pp] = t < Nkv ? *reinterpret_cast<const uint4*>(k + (bh * Nkv + t) * D + vc * 8) : make_uint4(0, 0, 0, 0);
     }
+    pdl_wait();  // kbar
     float kb[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) kb[i] = kbar[bh * D + vc * 8 + i];
@@ -317,6 +337,7 @@ __global__ void __launch_bounds__(kPrepThreads, 4)  // 4 CTAs per SM hide the lo
       const int t = kb_i * kTok + rs + pp * RPP;
       raw[pp] = t < Nkv ? *reinterpret_cast<const uint4*>(v + (bh * Nkv + t) * D + vc * 8) : make_uint4(0, 0, 0, 0);
     }
+    pdl_wait();  // sv
     float svc[8], rsv[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -471,6 +492,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     *abort_flag = 0;
     fence_mbarrier_init();
   }
+  pdl_wait();  // the prepass's codes, scales and q.kbar
   if (threadIdx.x < D) sv_smem[threadIdx.x] = p.sv[(size_t)bh_kv * D + threadIdx.x];
   if (warp == 8) {
     tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
@@ -800,29 +822,54 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
   }
 }
 
+// Launch that may start while the previous kernel on the stream finishes
+// (programmatic dependent launch; the kernel waits with pdl_wait before it
+// reads the previous kernel's output).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int D, bool F8>
 cudaError_t launch_q8_d(const Q8Launch& L, cudaStream_t stream) {
   const int nqb = L.p.nqb, nkb = L.p.nkb;
+  // the first launch waits for everything before it on the stream (a previous
+  // call's main kernel may still read the workspace this call rewrites)
   dim3 g1(nkb, L.Hkv, L.B);
   q8_kv_stats_kernel<D, F8><<<g1, kPrepThreads, 0, stream>>>(
       static_cast<const uint16_t*>(L.k), static_cast<const uint16_t*>(L.v), L.p.Nkv, nkb,
       L.ksum_part, L.vmax_part);
-  dim3 g2((unsigned)((long long)L.B * L.Hkv), D / 32);
-  q8_kv_final_kernel<D, F8><<<g2, 32 * kFinalSlices, 0, stream>>>(L.ksum_part, L.vmax_part, L.p.Nkv, nkb, L.kbar,
-                                              const_cast<float*>(L.p.sv));
-  const long long tiles = (long long)L.B * L.p.Hq * nqb + 2LL * L.B * L.Hkv * nkb;
-  q8_quantize_kernel<D, F8><<<(unsigned)tiles, kPrepThreads, 0, stream>>>(
-      static_cast<const uint16_t*>(L.q), static_cast<const uint16_t*>(L.k),
-      static_cast<const uint16_t*>(L.v), L.B, L.p.Hq, L.Hkv, L.p.Nq, L.p.Nkv, nqb, nkb, L.kbar,
-      L.p.sv, L.q8, L.k8, L.v8, const_cast<float*>(L.p.sq), const_cast<float*>(L.p.sk),
-      const_cast<float*>(L.p.qk));
   cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dim3 g2((unsigned)((long long)L.B * L.Hkv), D / 32);
+  e = launch_dependent(q8_kv_final_kernel<D, F8>, g2, dim3(32 * kFinalSlices), 0, stream,
+                       (const double*)L.ksum_part, (const float*)L.vmax_part, L.p.Nkv, nkb, L.kbar,
+                       const_cast<float*>(L.p.sv));
+  if (e != cudaSuccess) return e;
+  const long long tiles = (long long)L.B * L.p.Hq * nqb + 2LL * L.B * L.Hkv * nkb;
+  e = launch_dependent(q8_quantize_kernel<D, F8>, dim3((unsigned)tiles), dim3(kPrepThreads), 0, stream,
+                       static_cast<const uint16_t*>(L.q), static_cast<const uint16_t*>(L.k),
+                       static_cast<const uint16_t*>(L.v), L.B, L.p.Hq, L.Hkv, L.p.Nq, L.p.Nkv, nqb,
+                       nkb, (const float*)L.kbar, L.p.sv, L.q8, L.k8, L.v8,
+                       const_cast<float*>(L.p.sq), const_cast<float*>(L.p.sk),
+                       const_cast<float*>(L.p.qk));
   if (e != cudaSuccess || L.prepass_only) return e;
   e = max_dynamic_smem_once<attn_fwd_q8_kernel<D, F8>>(Q8Cfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(L.p.num_row_blocks, L.p.Hq, L.B);
-  attn_fwd_q8_kernel<D, F8><<<grid, kQ8Threads, Q8Cfg<D>::kSmemBytes, stream>>>(L.tq, L.tk, L.tv, L.to, L.p);
-  return cudaGetLastError();
+  return launch_dependent(attn_fwd_q8_kernel<D, F8>, grid, dim3(kQ8Threads), Q8Cfg<D>::kSmemBytes,
+                          stream, L.tq, L.tk, L.tv, L.to, L.p);
 }
 
 }  // namespace

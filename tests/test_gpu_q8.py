@@ -177,6 +177,14 @@ def test_q8_forward_workloads(name):
     _check_fwd(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.causal, w.seed, w.dist, n_rows=w.oracle_rows)
 
 
+def test_fp8qk_forward_8k_outlier_workload():
+    """The FP8 Q K^T variant on the bench's 8k outlier workload (sampled rows):
+    within the per-element bound around its own method's result."""
+    w = WORKLOADS["q8_8k_outlier"]
+    _check_fwd(w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.causal, w.seed, w.dist, n_rows=w.oracle_rows,
+               qk_format="fp8")
+
+
 @pytest.mark.slow
 def test_q8_forward_every_row_8k_outlier():
     """Every row of the 8-bit 8k outlier workload against the exact fp64 oracle
