@@ -232,7 +232,7 @@ def time_graph_replays(step, steps: int, flush):
 
 
 def bench_workload(w: Workload, steps: int, warmup: int, world: int, rank: int, lib_mod,
-                   graph: bool = False):
+                   graph: bool = False, qk_format: str = "int8"):
     import torch
     wr = rank_workload(w, rank)
     q, k, v = make_qkv(wr.B, wr.Hq, wr.Hkv, wr.Nq, wr.Nkv, wr.d, wr.seed, wr.dist)
@@ -251,7 +251,8 @@ def bench_workload(w: Workload, steps: int, warmup: int, world: int, rank: int, 
                          dtype=torch.uint8, device="cuda")
 
         def step():
-            lib_mod.attn_fwd_q8(qd, kd, vd, causal=w.causal, workspace=ws, out=o, lse=lse)
+            lib_mod.attn_fwd_q8(qd, kd, vd, causal=w.causal, workspace=ws, out=o, lse=lse,
+                                qk_format=qk_format)
     elif w.path == "splitkv":
         need = int(lib_mod.lib().attn_fwd_splitkv_workspace_size(wr.B, wr.Hq, wr.Hkv, wr.Nq, wr.Nkv,
                                                                    wr.d, 0))
@@ -485,7 +486,7 @@ def run_ours(args):
     # warm the kernel and sample clocks only over the timed region
     res = None
     clocks.start()
-    res = bench_workload(w, args.steps, args.warmup, world, rank, attn)
+    res = bench_workload(w, args.steps, args.warmup, world, rank, attn, qk_format=args.qk_format)
     clk = clocks.stop()
     ms = res["total_ms"] / args.steps
     value = aggregate_tflops(w.flops, world, ms)
@@ -568,9 +569,11 @@ def run_ours(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16" if w.path != "q8" else "int8 QK^T + e4m3 PV (fp32 accumulation)",
+            "dtype": "bf16" if w.path != "q8" else
+                     f"{'int8' if args.qk_format == 'int8' else 'e4m3'} QK^T + e4m3 PV (fp32 accumulation)",
             "data": "synthetic (seeded torch CPU randn -> bf16; outlier-K offsets per head/channel)",
-            "config": workload_config(w, res["l2"]),
+            "config": ({**workload_config(w, res["l2"]), "qk_format": args.qk_format} if w.path == "q8"
+                       else workload_config(w, res["l2"])),
             "frac_of_bf16_peak": round(value / world / peaks["bf16"], 4),
             "roofline": {"bound": "tensor", "achieved": round(per_launch_tflops, 2),
                          "peak": peaks["bf16"] * (2 if w.path == "q8" else 1), "unit": "TFLOP/s",
@@ -582,7 +585,10 @@ def run_ours(args):
                                    "attn_fwd_q8 (3 prepass kernels + main kernel)",
                          "algorithmic_min_bytes": w.min_hbm_bytes},
             "e2e": e2e,
-            "gpu_launches": args.steps,
+            # per call: 1 kernel; the 8-bit path 3 prepass kernels + main; split keys partial + merge
+            "gpu_launches": args.steps * (4 if w.path == "q8" else
+                                          (2 if w.path == "splitkv" and attn.splitkv_num_splits(
+                                              w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d) > 1 else 1)),
             "clocks": clk,
             "cpu_baseline": cpu,
             "other_workloads": extras,
@@ -750,6 +756,8 @@ def main():
                     help="only the device-timed leg (for profiling runs): no e2e, CPU or extra legs")
     ap.add_argument("--direction", default="fwd", choices=["fwd", "bwd"],
                     help="bwd: time only the backward of --workload (one JSON line)")
+    ap.add_argument("--qk-format", default="int8", choices=["int8", "fp8"],
+                    help="8-bit workloads: INT8 Q K^T after K smoothing, or FP8 e4m3 Q K^T with block scales")
     ap.add_argument("--shard", default="batch", choices=["batch", "kv"],
                     help="kv: split the keys of --workload over the ranks (key-sharded forward, "
                          "partial -> NCCL all-gather -> merge; default workload kvcache_128k_q128)")
