@@ -214,14 +214,19 @@ ATTN_API attn_status_t attn_fwd_host(const void* q_host, const void* k_host, con
  * Nkv tokens (lossless by the shift invariance of softmax; LSE is corrected
  * back), Q and the smoothed K are quantised to INT8 with one fp32 scale per
  * 128-token block, V to FP8 e4m3 with one fp32 scale per channel; S = Q8 K8^T
- * runs on INT8 tensor cores (s32 accumulation), P is encoded as e4m3(p * 448)
- * and P8 V8 runs on FP8 tensor cores (fp32 accumulation).
+ * runs on INT8 tensor cores (s32 accumulation), P is encoded as
+ * e4m3(2^(t - m_ref) * 448 / 16) against a reference maximum m_ref that lags
+ * the row maximum by at most 2^4 (so O is rescaled only when it is overtaken
+ * by more), and P8 V8 runs on FP8 tensor cores (fp32 accumulation).
  *   inputs/outputs  as attn_fwd (bf16 q, k, v; bf16 o; fp32 lse)
  *   workspace       device, caller-owned, 16-byte aligned, at least
  *                   attn_fwd_q8_workspace_size() bytes; holds the quantised
  *                   tensors and scales (its contents after the call are the
  *                   prepass results, see attn_q8_workspace_offsets)
- * Four launches on `stream` (three prepass kernels, one main kernel).
+ * Four launches on `stream` (three prepass kernels, one main kernel); the
+ * last three are dependent launches that may start while their predecessor
+ * finishes and wait on the device for its results, the first waits for all
+ * earlier work on `stream`.
  * Errors: as attn_fwd, plus ATTN_ERR_WORKSPACE for a NULL, misaligned or too
  * small workspace.
  */
@@ -239,7 +244,8 @@ ATTN_API attn_status_t attn_fwd_q8(const void* q, const void* k, const void* v, 
  * FP8 tensor cores with fp32 accumulation; P and V exactly as in attn_fwd_q8.
  * It is the comparison point for INT8 with K smoothing on channels with
  * outliers. Same arguments, workspace and errors as attn_fwd_q8 (the workspace
- * regions hold e4m3 codes for Q and K, kbar and q.kbar are zero).
+ * regions hold e4m3 codes for Q and K, kbar and q.kbar are zero; its
+ * statistics kernel reads V only).
  * attn_fp8_prepass runs only its three prepass launches.
  */
 ATTN_API attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
