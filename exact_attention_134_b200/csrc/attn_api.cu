@@ -265,8 +265,10 @@ attn_status_t run_fwd_varlen(const void* q, const void* k, const void* v, void* 
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.causal = causal;
+  // grid x: the units of all sequences, at most one item per sequence without one
+  // (packed_unit); max_seqlen_q is not needed for it
   const int rows = d == 256 ? attn_sm100::fwd_rows_per_cta_d256() : attn_sm100::fwd_rows_per_cta();
-  p.num_row_blocks = (max_seqlen_q + rows - 1) / rows;
+  p.num_row_blocks = total_q / rows + num_seqs;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = (unsigned long long)g_timeout_ns.load();
   if (d == 256) return cuda_status(attn_sm100::launch_fwd_d256(tk, tv, q, p, stream));

@@ -23,8 +23,9 @@
 // was issued before it (tcgen05 MMAs from one thread execute in order). O is
 // rescaled only when a row's running maximum moves by more than 2^8, and only
 // then does the softmax wait for PV(j-1).
-// VL = true: packed variable-length sequences [total, H, d] (grid z = sequence,
-// rows from cu_seqlens, per-sequence bottom-right causal mask). A K/V tile that
+// VL = true: packed variable-length sequences [total, H, d] (grid x = query
+// head, (y, z) = the 128-row units of all sequences, see packed_unit; rows
+// from cu_seqlens, per-sequence bottom-right causal mask). A K/V tile that
 // runs past its sequence reads the next sequence's rows (or the map's zero
 // fill past the end); those columns are masked to -inf, so P = 0 there.
 #include <cuda.h>
@@ -116,7 +117,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   grouped_heavy_first(VL ? 0 : p.lpt_group, ux, hq, b);
   int Lq = p.Nq, Lk = p.Nkv, q_start = 0, k_start = 0;
   if (VL) {
-    const int sq = blockIdx.z;
+    // grid (head, item % rows, item / rows): consecutive CTAs are the heads of
+    // one unit, and a sequence's units come heaviest first
+    hq = blockIdx.x;
+    const int item = (int)(blockIdx.y + (long long)blockIdx.z * gridDim.y);
+    const int sq = packed_unit(p.cu_q, p.B, p.Nq, kBM, item, ux);
     q_start = min(max(p.cu_q[sq], 0), p.Nq);
     Lq = min(max(p.cu_q[sq + 1], q_start), p.Nq) - q_start;
     k_start = min(max(p.cu_k[sq], 0), p.Nkv);
@@ -124,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     b = 0;
   }
   const int nrb = (Lq + kBM - 1) / kBM;
-  if (ux >= nrb) return;  // this sequence has fewer rows (the whole CTA leaves)
+  if (ux < 0 || ux >= nrb) return;  // no unit for this item (the whole CTA leaves)
   const int row_block = p.causal ? (nrb - 1 - ux) : ux;
   const int hk = hq / (p.Hq / p.Hkv);
   const int q0 = row_block * kBM;
@@ -390,8 +395,11 @@ cudaError_t launch_d256(const CUtensorMap& tk, const CUtensorMap& tv, const void
                         const FwdParams& p, cudaStream_t stream) {
   cudaError_t e = max_dynamic_smem_once<attn_fwd_d256_kernel<VL>>(kSmemBytes);
   if (e != cudaSuccess) return e;
-  // packed: grid x covers the longest sequence (p.num_row_blocks), z = sequence
-  dim3 grid(VL ? p.num_row_blocks : (p.Nq + kBM - 1) / kBM, p.Hq, p.B);
+  dim3 grid((p.Nq + kBM - 1) / kBM, p.Hq, p.B);
+  if (VL) {  // x = head, the units of all sequences over y (at most 65535) and z
+    const unsigned items = (unsigned)p.num_row_blocks, gy = items < 65535u ? items : 65535u;
+    grid = dim3((unsigned)p.Hq, gy, (items + gy - 1) / gy);
+  }
   attn_fwd_d256_kernel<VL><<<grid, kThreads, kSmemBytes, stream>>>(tk, tv, q, p);
   return cudaGetLastError();
 }

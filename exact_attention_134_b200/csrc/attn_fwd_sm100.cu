@@ -120,9 +120,11 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
 }
 
 // VL = false: dense [B, H, N, d] tensors, one grid z-slice per batch entry.
-// VL = true : packed variable-length sequences [total, H, d]; grid z = sequence,
-//             its query/key rows come from cu_seqlens; O and LSE are stored
-//             row by row (a TMA box could cross into the next sequence).
+// VL = true : packed variable-length sequences [total, H, d]; grid x = query
+//             head, (y, z) run over the units of all sequences (packed_unit);
+//             the query/key rows of a unit's sequence come from cu_seqlens; O
+//             and LSE are stored row by row (a TMA box could cross into the
+//             next sequence).
 // PART = true (dense only): a partial result over key ranges — grid z = batch
 //             entry x range, fp32 O rows and LSE per range, the causal mask
 //             aligned to the end of the full key sequence (p.kv_tail keys
@@ -162,8 +164,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   int ux, uy, uz;
   grouped_heavy_first((!VL && !PART) ? p.lpt_group : 0, ux, uy, uz);
   int Lq = p.Nq, Lk = p.Nkv, q_start = 0, k_start = 0;
+  constexpr int kUnitRows = PAIR ? kBM : 2 * kBM;  // query rows of a work unit
   if (VL) {
-    const int sq = blockIdx.z;
+    // grid (head, item % rows, item / rows): consecutive CTAs are the heads of
+    // one unit, and a sequence's units come heaviest first
+    uy = blockIdx.x;
+    const int item = (int)(blockIdx.y + (long long)blockIdx.z * gridDim.y);
+    const int sq = packed_unit(p.cu_q, p.B, p.Nq, kUnitRows, item, ux);
     q_start = min(max(p.cu_q[sq], 0), p.Nq);
     Lq = min(max(p.cu_q[sq + 1], q_start), p.Nq) - q_start;
     k_start = min(max(p.cu_k[sq], 0), p.Nkv);
@@ -173,10 +180,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_start = ((int)blockIdx.z % p.num_splits) * p.kv_chunk;  // < Nkv: only non-empty ranges are launched
     Lk = min(p.Nkv - k_start, p.kv_chunk);
   }
-  constexpr int kUnitRows = PAIR ? kBM : 2 * kBM;  // query rows of a work unit
   constexpr int kTileRowStep = PAIR ? 0 : kBM;    // first row of tile 1 - of tile 0
   const int nrb = (Lq + kUnitRows - 1) / kUnitRows;
-  if (ux >= nrb) return;  // this sequence has fewer rows (the whole CTA leaves)
+  if (ux < 0 || ux >= nrb) return;  // no unit for this item (the whole CTA leaves)
   const int row_block = p.causal ? (nrb - 1 - ux) : ux;
   const int hq = PAIR ? 2 * uy : uy;  // query head of tile 0
   const int b = VL ? 0 : (PART ? uz / p.num_splits : uz);
@@ -561,8 +567,13 @@ static cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, co
                                 const CUtensorMap& to, const FwdParams& p, cudaStream_t stream) {
   cudaError_t e = max_dynamic_smem_once<attn_fwd_bf16_kernel<D, VL, PART, PAIR>>(smem_bytes<D>());
   if (e != cudaSuccess) return e;
-  // varlen: B = number of sequences; head pairs: Hq / 2 units of 128 rows
+  // head pairs: Hq / 2 units of 128 rows; packed sequences: x = head, the units
+  // of all sequences over y (at most 65535) and z
   dim3 grid(p.num_row_blocks, PAIR ? p.Hq / 2 : p.Hq, p.B * p.num_splits);
+  if (VL) {
+    const unsigned items = (unsigned)p.num_row_blocks, gy = items < 65535u ? items : 65535u;
+    grid = dim3((unsigned)p.Hq, gy, (items + gy - 1) / gy);
+  }
   attn_fwd_bf16_kernel<D, VL, PART, PAIR><<<grid, kThreads, smem_bytes<D>(), stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }

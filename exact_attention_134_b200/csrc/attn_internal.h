@@ -28,6 +28,30 @@ cudaError_t max_dynamic_smem_once(int bytes) {
   return e;
 }
 
+#ifdef __CUDACC__
+// Packed sequences: maps work item i of a grid row to a sequence and a unit
+// (a block of U rows) of it, with no row per sequence of the longest one.
+// Sequence s's ceil(L_s / U) units occupy items [v(s), v(s) + ceil(L_s / U)),
+// v(s) = floor(off[s] / U) + s (off = its row offsets, clamped to [0, total]);
+// these ranges are disjoint and increase with s, and items
+// 0 .. floor(total / U) + num_seqs - 1 cover them all, so a grid row of that
+// many items has at most one item per sequence without a unit. Returns s (the
+// largest with v(s) <= i, by binary search) and sets `rank` = i - v(s), the
+// unit index within the sequence (>= its unit count for an item without one).
+__device__ __forceinline__ int packed_unit(const int* off, int num_seqs, int total, int U, int i,
+                                           int& rank) {
+  auto v = [&](int s) { return min(max(off[s], 0), total) / U + s; };
+  int lo = 0, hi = num_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (v(mid) <= i) lo = mid;
+    else hi = mid - 1;
+  }
+  rank = i - v(lo);
+  return lo;
+}
+#endif
+
 // Kernel parameters of the bf16 forward (tensor maps are passed separately).
 struct FwdParams {
   void* o;                        // bf16 [B, Hq, Nq, d]
@@ -37,7 +61,7 @@ struct FwdParams {
   const int* cu_k;                //                   key row offsets [B + 1]
   int B, Nq, Nkv, Hq, Hkv;        // packed: B = sequences, Nq / Nkv = total rows
   int causal;
-  int num_row_blocks;             // ceil(Nq / rows per work unit); packed: of the longest sequence
+  int num_row_blocks;             // ceil(Nq / rows per work unit); packed: floor(total_q / rows) + sequences
   float scale_log2;               // scale * log2(e)
   unsigned long long timeout_ns;  // budget of every pipeline wait
   // Partial results over key ranges (dense tensors only; see attn_fwd_partial):

@@ -94,8 +94,9 @@ ATTN_API attn_status_t attn_fwd(const void* q, const void* k, const void* v, voi
  *   cu_seqlens_q/k device, int32 [num_seqs + 1], non-decreasing, starting at 0
  *                  and ending at total_q / total_k (caller's responsibility;
  *                  offsets outside [0, total] are clamped, never followed)
- *   max_seqlen_q   >= the longest query sequence (sizes the grid; rows beyond
- *                  it are not computed)
+ *   max_seqlen_q   > 0, kept for interface compatibility: the grid holds one
+ *                  CTA per 256-row unit (128 at d = 256) of every sequence,
+ *                  sized from total_q and num_seqs, so every row is computed
  *   d              64, 96, 128 or 256 (the head dimension up to 256 of the same
  *                  page's section "FlashAttention-2 (2023)")
  * Allocates nothing; one kernel launch on `stream`.
