@@ -89,6 +89,10 @@ VARLEN = [
     ([64, 200, 513], [1000, 200, 700], 4, 2, 256, True),     # head dim 256, prefill with a cache
     ([300, 50, 5], [100, 0, 5], 2, 2, 256, True),            # head dim 256, Lq > Lk, an empty key set
     ([700, 0, 33], [700, 40, 33], 2, 2, 256, False),         # head dim 256, an empty query sequence
+    # one long prompt among many tiny and empty ones: work items map to units
+    # across sequence boundaries, with empty items between them
+    ([700] + [0, 1, 2, 3, 5, 1, 0, 4] * 5 + [257], None, 4, 2, 128, True),
+    ([3, 0, 300] + [1, 0, 2] * 6 + [129], None, 2, 1, 256, True),
 ]
 
 
