@@ -503,9 +503,10 @@ attn_status_t run_bwd(const void* q, const void* k, const void* v, const void* o
     // a group's Q, dO (bf16) and dQ accumulator (fp32) within 32 MiB
     const long long per_kv_head = 8LL * Nq * d * (Hq / Hkv);
     p.lpt_group = (int)std::min((long long)B * Hkv, std::max(1LL, (32LL << 20) / per_kv_head));
-  } else if (causal && vl && max_k > 128) {
-    p.lpt_group = Hkv;  // the kv heads of one sequence
   }
+  // packed sequences: the grid is (kv head, key units of all sequences), so the
+  // kv heads of one unit run together and a sequence's heavy first keys first
+  p.num_seqs = vl ? B : 0;
   L.post.dq_acc = acc;
   L.post.dq = dq;
   L.post.cu_q = cu_q;

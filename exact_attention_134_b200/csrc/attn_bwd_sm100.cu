@@ -194,10 +194,13 @@ __device__ __forceinline__ void store_row(uint32_t t_row, float mul, uint16_t* d
 }
 
 // VL = false: dense [B, H, N, d] tensors, grid z = batch entry.
-// VL = true : packed variable-length sequences [total, H, d], grid z =
-//             sequence; rows past a sequence's end (the next sequence's) are
-//             loaded but contribute nothing: their keys are masked and their
-//             queries carry LSE_2 = +inf (P = dS = 0).
+// VL = true : packed variable-length sequences [total, H, d]; grid x = kv
+//             head, (y, z) run over the 128-key units of all sequences
+//             (packed_unit: consecutive CTAs are the kv heads of one unit, a
+//             sequence's first, heaviest key blocks come first); rows past a
+//             sequence's end (the next sequence's) are loaded but contribute
+//             nothing: their keys are masked and their queries carry
+//             LSE_2 = +inf (P = dS = 0).
 template <int D, bool VL>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -216,7 +219,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // seen by the most queries) across groups of p.lpt_group (kv head, batch or
   // sequence) pairs whose Q, dO and dQ accumulator stay in L2.
   int kb, hk, b;  // b: batch entry, or sequence (VL)
-  grouped_heavy_first(p.lpt_group, kb, hk, b);
+  grouped_heavy_first(VL ? 0 : p.lpt_group, kb, hk, b);
+  if (VL) {
+    hk = blockIdx.x;
+    const int item = (int)(blockIdx.y + (long long)blockIdx.z * gridDim.y);
+    b = packed_unit(p.cu_k, p.num_seqs, p.Nkv, kBK, item, kb);
+  }
   const int G = p.Hq / p.Hkv;
   const int k0 = kb * kBK;
   int Lq = p.Nq, Lk = p.Nkv, q_start = 0, k_start = 0;
@@ -227,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Lq = min(min(max(p.cu_q[b + 1], q_start), p.Nq) - q_start, p.nq_pad);
     k_start = min(max(p.cu_k[b], 0), p.Nkv);
     Lk = min(max(p.cu_k[b + 1], k_start), p.Nkv) - k_start;
-    if (k0 >= Lk) return;  // this sequence has fewer keys (the whole CTA leaves)
+    if (kb < 0 || k0 >= Lk) return;  // no key unit for this item (the whole CTA leaves)
   }
   // row of key k0 + r in dK / dV, and TMA coordinates of K/V and Q/dO tiles
   auto kv_row_off = [&](int r) -> size_t {
@@ -724,6 +732,10 @@ cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
   e = max_dynamic_smem_once<attn_bwd_main_kernel<D, VL>>(BwdCfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((L.max_kv + kBK - 1) / kBK, L.main.Hkv, L.B);
+  if (VL) {  // x = kv head, the key units of all sequences over y (at most 65535) and z
+    const unsigned items = (unsigned)(L.main.Nkv / kBK + L.B), gy = items < 65535u ? items : 65535u;
+    grid = dim3((unsigned)L.main.Hkv, gy, (items + gy - 1) / gy);
+  }
   attn_bwd_main_kernel<D, VL><<<grid, kThreads, BwdCfg<D>::kSmemBytes, stream>>>(L.tq, L.tk, L.tv, L.tdo,
                                                                               L.main);
   e = cudaGetLastError();

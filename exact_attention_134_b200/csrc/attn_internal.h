@@ -135,6 +135,7 @@ struct BwdParams {
   // Dense causal: dispatch order groups of (batch, kv head) pairs, key blocks
   // heaviest first across a group (0 = the grid's own order).
   int lpt_group;
+  int num_seqs;                   // packed sequences: their count (else unused)
 };
 
 struct BwdPreParams {
