@@ -38,8 +38,8 @@ cudaError_t max_dynamic_smem_once(int bytes) {
 // many items has at most one item per sequence without a unit. Returns s (the
 // largest with v(s) <= i, by binary search) and sets `rank` = i - v(s), the
 // unit index within the sequence (>= its unit count for an item without one).
-__device__ __forceinline__ int packed_unit(const int* off, int num_seqs, int total, int U, int i,
-                                           int& rank) {
+__host__ __device__ __forceinline__ int packed_unit(const int* off, int num_seqs, int total, int U,
+                                                    int i, int& rank) {
   auto v = [&](int s) { return min(max(off[s], 0), total) / U + s; };
   int lo = 0, hi = num_seqs - 1;
   while (lo < hi) {
