@@ -74,6 +74,66 @@ def _traffic_from_profile(workload: str):
     return None if per is None else per.get("dram_bytes_per_launch")
 
 
+class NvmlClockSampler:
+    """SM clock and throttle reasons read through NVML (read-only queries) by a
+    thread polling about every millisecond, so even a timed region of a few
+    milliseconds is sampled. The GPU is found by the CUDA device's PCI bus id."""
+
+    def __init__(self, device_index: int):
+        import pynvml
+        import torch
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        prop = torch.cuda.get_device_properties(device_index)
+        bus = f"{prop.pci_domain_id:08x}:{prop.pci_bus_id:02x}:{prop.pci_device_id:02x}.0"
+        self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.samples = []
+        self.stop_event = threading.Event()
+
+    def start(self):
+        self.thread = threading.Thread(target=self._poll, daemon=True)
+        self.thread.start()
+
+    def _poll(self):
+        nv = self.nv
+        while True:
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((float(mhz), int(reasons)))
+            except Exception:  # a failed read is skipped, not fatal
+                pass
+            if self.stop_event.wait(0.001):
+                return
+
+    def stop(self):
+        self.stop_event.set()
+        self.thread.join(timeout=5)
+        nv = self.nv
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        try:
+            nv.nvmlShutdown()
+        except Exception:
+            pass
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"], "source": "nvml"}
+        reasons = sorted(n for n, b in bits.items() if any(r & b for _, r in self.samples))
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
+
+
+def clock_sampler(device_index: int):
+    """NVML sampler when NVML answers for this device, else nvidia-smi."""
+    try:
+        return NvmlClockSampler(device_index)
+    except Exception:
+        return ClockSampler(device_index)
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples during the timed region."""
 
@@ -481,7 +541,7 @@ def run_ours(args):
     world, rank, local = _dist_setup()
     peaks = _peaks()
     w = WORKLOADS[args.workload]
-    clocks = ClockSampler(local)
+    clocks = clock_sampler(local)
     attn.lib()
     # warm the kernel and sample clocks only over the timed region
     res = None
@@ -640,7 +700,7 @@ def run_kv_shard(args):
     def step():
         return attention_kv_sharded(qd, kd, vd, n_keys, causal=w.causal)
 
-    clocks = ClockSampler(local)
+    clocks = clock_sampler(local)
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
