@@ -347,9 +347,11 @@ ATTN_API attn_status_t attn_bwd(const void* q, const void* k, const void* v, con
  * gradients of attn_fwd_varlen: q, o, dout, dq [total_q, Hq, d]; k, v, dk, dv
  * [total_k, Hkv, d]; lse fp32 [Hq, total_q] as attn_fwd_varlen writes it;
  * cu_seqlens_q / cu_seqlens_k int32 device arrays [num_seqs + 1] (sequence s
- * owns rows cu[s] .. cu[s+1]); max_seqlen_q / max_seqlen_k must bound every
- * sequence's rows (they size the grid and the workspace; rows beyond them are
- * not computed, and nothing outside the buffers is touched). Causal masks are
+ * owns rows cu[s] .. cu[s+1]); max_seqlen_q must bound every sequence's query
+ * rows (it sizes the workspace; query rows beyond it are not computed, and
+ * nothing outside the buffers is touched); max_seqlen_k > 0 is kept for
+ * interface compatibility (the grid holds one CTA per 128-key unit of every
+ * sequence, sized from total_k and num_seqs). Causal masks are
  * aligned to the bottom right of each sequence. Rows of dk / dv that no
  * query sees are written as 0. Workspace: attn_bwd_varlen_workspace_size()
  * bytes (fp32 dQ accumulator with every sequence padded to max_seqlen_q
