@@ -675,9 +675,9 @@ def run_kv_shard(args):
     """Key-sharded forward of one long-context workload over the ranks (strong
     scaling: the total work is fixed). Each step runs attn_fwd_partial on the
     rank's key range (split over CTAs and merged on the device when the range's
-    grid alone would leave SMs idle), two NCCL all-gathers of the fp32 partials
-    and the merge (kv_shard.attention_kv_sharded); time = max over ranks of the
-    CUDA-event time. One JSON line from rank 0."""
+    grid alone would leave SMs idle), one NCCL all-gather of the packed fp32
+    partials and the merge (kv_shard.attention_kv_sharded); time = max over
+    ranks of the CUDA-event time. One JSON line from rank 0."""
     import datetime
     import torch
     import torch.distributed as dist
@@ -718,7 +718,7 @@ def run_kv_shard(args):
     total_ms, any_err = float(t[0]), float(t[1])
     ms = total_ms / args.steps
     value = w.flops / (ms * 1e-3) / 1e12
-    exchange = world * w.B * w.Hq * w.Nq * (w.d + 1) * 4
+    exchange = world * attn.partial_packed_floats(w.B, w.Hq, w.Nq, w.d) * 4  # fp32 O and LSE, packed
     # partial (+ the range's own merge when it is split) + the final merge
     local_splits = attn.splitkv_num_splits(w.B, w.Hq, w.Hkv, w.Nq, ks.shape[2], w.d)
     launches_per_step = 3 if local_splits > 1 else 2
@@ -732,7 +732,7 @@ def run_kv_shard(args):
                           "shard": "kv"},
                "frac_of_bf16_peak": round(value / world / peaks["bf16"], 4),
                "exchange_bytes_per_rank": exchange,
-               "collectives_per_step": "2 NCCL all-gathers (fp32 O and LSE partials)",
+               "collectives_per_step": "1 NCCL all-gather (fp32 O and LSE partials, packed)",
                "local_key_ranges": local_splits,
                "gpu_launches": launches_per_step * args.steps,
                "clocks": clk, "device_status_error": bool(any_err)}

@@ -47,6 +47,8 @@ _SIGNATURES = {
     "attn_fwd_varlen": (_c_int, [_vp] * 7 + [_c_int] * 8 + [_c_float, _vp]),
     "attn_fwd_partial": (_c_int, [_vp] * 5 + [_c_int] * 7 + [_c_float, _c_int, _vp]),
     "attn_merge_partials": (_c_int, [_vp, _vp] + [_c_int] * 5 + [_vp, _vp, _vp]),
+    "attn_partial_packed_floats": (ctypes.c_longlong, [_c_int] * 4),
+    "attn_merge_partials_packed": (_c_int, [_vp] + [_c_int] * 5 + [_vp, _vp, _vp]),
     "attn_fwd_splitkv_num_splits": (_c_int, [_c_int] * 7),
     "attn_fwd_splitkv_workspace_size": (_sz, [_c_int] * 7),
     "attn_fwd_splitkv": (_c_int, [_vp] * 5 + [_c_int] * 7 + [_c_float, _c_int, _vp, _sz, _vp]),
@@ -207,6 +209,32 @@ def merge_partials(o_parts, lse_parts, out=None, lse=None):
     st = lib().attn_merge_partials(o_parts.data_ptr(), lse_parts.data_ptr(), S, B, Hq, Nq, d,
                                    out.data_ptr(), lse.data_ptr(), _stream_handle(o_parts.device))
     _check(st, "attn_merge_partials")
+    return out, lse
+
+
+def partial_packed_floats(B, Hq, Nq, d) -> int:
+    """Floats per part of the packed partial layout: fp32 O [B, Hq, Nq, d], then
+    fp32 LSE [B, Hq, Nq], padded to a multiple of 4."""
+    return int(lib().attn_partial_packed_floats(B, Hq, Nq, d))
+
+
+def merge_partials_packed(parts, B, Hq, Nq, d, out=None, lse=None):
+    """merge_partials over parts packed one after another (fp32 cuda
+    [S, partial_packed_floats(B, Hq, Nq, d)], each part = O then LSE), the layout
+    one all-gather of every rank's packed partial produces.
+    -> (o bf16 [B, Hq, Nq, d], lse fp32 [B, Hq, Nq])."""
+    import torch
+    stride = partial_packed_floats(B, Hq, Nq, d)
+    if parts.dtype != torch.float32 or not parts.is_cuda or not parts.is_contiguous() or \
+            parts.dim() != 2 or parts.shape[1] != stride:
+        raise ValueError(f"parts must be a contiguous fp32 CUDA tensor [S, {stride}]")
+    if out is None:
+        out = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=parts.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=parts.device)
+    st = lib().attn_merge_partials_packed(parts.data_ptr(), parts.shape[0], B, Hq, Nq, d,
+                                          out.data_ptr(), lse.data_ptr(), _stream_handle(parts.device))
+    _check(st, "attn_merge_partials_packed")
     return out, lse
 
 

@@ -627,6 +627,25 @@ attn_status_t attn_merge_partials(const float* o_parts, const float* lse_parts, 
                                               static_cast<cudaStream_t>(stream)));
 }
 
+long long attn_partial_packed_floats(int B, int Hq, int Nq, int d) {
+  if (B <= 0 || Hq <= 0 || Nq <= 0 || d <= 0) return 0;
+  const long long rows = (long long)B * Hq * Nq;
+  return (rows * d + rows + 3) / 4 * 4;
+}
+
+attn_status_t attn_merge_partials_packed(const float* parts, int num_parts, int B, int Hq, int Nq,
+                                         int d, void* o, float* lse, void* stream) {
+  if (!parts || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (num_parts <= 0 || B <= 0 || Hq <= 0 || Nq <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 96 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(parts) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_ALIGNMENT;
+  const long long rows = (long long)B * Hq * Nq;
+  const long long stride = attn_partial_packed_floats(B, Hq, Nq, d);
+  return cuda_status(attn_sm100::launch_merge(parts, parts + rows * d, num_parts, rows, d, o, lse,
+                                              static_cast<cudaStream_t>(stream), false, stride,
+                                              stride));
+}
+
 int attn_fwd_splitkv_num_splits(int B, int Hq, int Hkv, int Nq, int Nkv, int d, int num_splits) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Nq <= 0 || Nkv <= 0 || d <= 0) return 0;
   return plan_splits(B, Hq, Hkv, Nq, Nkv, d, num_splits).splits;

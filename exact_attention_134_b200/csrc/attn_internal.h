@@ -187,11 +187,13 @@ int fwd_rows_per_cta();
 int fwd_rows_per_cta_paired();
 
 // O = sum_s exp(LSE_s - LSE) O_s, LSE = ln sum_s exp(LSE_s) over num_parts
-// partial results [num_parts, rows, d] fp32 / [num_parts, rows] fp32;
-// writes O [rows, d] (bf16, or fp32 with o_fp32) and fp32 LSE [rows].
+// partial results: part s's fp32 O rows [rows, d] at o_parts + s * o_stride and
+// its fp32 LSE [rows] at lse_parts + s * lse_stride (strides in floats; <= 0:
+// stacked, rows * d and rows); writes O [rows, d] (bf16, or fp32 with o_fp32)
+// and fp32 LSE [rows].
 cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int num_parts,
                          long long rows, int d, void* o, float* lse, cudaStream_t stream,
-                         bool o_fp32 = false);
+                         bool o_fp32 = false, long long o_stride = 0, long long lse_stride = 0);
 
 // Head dim 256, dense tensors or (p.cu_q set) packed sequences: K/V tensor maps
 // with 64-row boxes; Q is read directly from global memory.

@@ -33,20 +33,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
 template <int D, bool F32>
 __global__ void __launch_bounds__(D / 4 * kRowsPerCta)
     attn_merge_kernel(const float* __restrict__ o_parts, const float* __restrict__ lse_parts,
-                      int num_parts, long long rows, void* __restrict__ o,
-                      float* __restrict__ lse) {
+                      int num_parts, long long rows, long long o_stride, long long lse_stride,
+                      void* __restrict__ o, float* __restrict__ lse) {
   constexpr int kT = D / 4;  // threads per row
   const int c4 = threadIdx.x % kT;
   const long long r = (long long)blockIdx.x * kRowsPerCta + threadIdx.x / kT;
   if (r >= rows) return;
   float m = -INFINITY;
-  for (int s = 0; s < num_parts; ++s) m = fmaxf(m, lse_parts[(size_t)s * rows + r]);
+  // part s: O rows at o_parts + s * o_stride, LSE at lse_parts + s * lse_stride (floats)
+  for (int s = 0; s < num_parts; ++s) m = fmaxf(m, lse_parts[(size_t)s * lse_stride + r]);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float total = 0.0f;
   if (m != -INFINITY) {
     for (int s = 0; s < num_parts; ++s) {
-      const float w = expf(lse_parts[(size_t)s * rows + r] - m);  // 0 for a -inf part
-      const float4 x = reinterpret_cast<const float4*>(o_parts + ((size_t)s * rows + r) * D)[c4];
+      const float w = expf(lse_parts[(size_t)s * lse_stride + r] - m);  // 0 for a -inf part
+      const float4 x = reinterpret_cast<const float4*>(o_parts + (size_t)s * o_stride + (size_t)r * D)[c4];
       acc.x = fmaf(w, x.x, acc.x);
       acc.y = fmaf(w, x.y, acc.y);
       acc.z = fmaf(w, x.z, acc.z);
@@ -69,15 +70,16 @@ __global__ void __launch_bounds__(D / 4 * kRowsPerCta)
 
 template <int D>
 cudaError_t launch_merge_d(const float* o_parts, const float* lse_parts, int num_parts,
-                           long long rows, void* o, float* lse, bool o_fp32, cudaStream_t stream) {
+                           long long rows, long long o_stride, long long lse_stride, void* o,
+                           float* lse, bool o_fp32, cudaStream_t stream) {
   const long long blocks = (rows + kRowsPerCta - 1) / kRowsPerCta;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   if (o_fp32)
     attn_merge_kernel<D, true><<<(unsigned)blocks, D / 4 * kRowsPerCta, 0, stream>>>(
-        o_parts, lse_parts, num_parts, rows, o, lse);
+        o_parts, lse_parts, num_parts, rows, o_stride, lse_stride, o, lse);
   else
     attn_merge_kernel<D, false><<<(unsigned)blocks, D / 4 * kRowsPerCta, 0, stream>>>(
-        o_parts, lse_parts, num_parts, rows, o, lse);
+        o_parts, lse_parts, num_parts, rows, o_stride, lse_stride, o, lse);
   return cudaGetLastError();
 }
 
@@ -85,12 +87,14 @@ cudaError_t launch_merge_d(const float* o_parts, const float* lse_parts, int num
 
 cudaError_t launch_merge(const float* o_parts, const float* lse_parts, int num_parts,
                          long long rows, int d, void* o, float* lse, cudaStream_t stream,
-                         bool o_fp32) {
+                         bool o_fp32, long long o_stride, long long lse_stride) {
+  if (o_stride <= 0) o_stride = rows * d;  // parts stacked: [num_parts, rows, d]
+  if (lse_stride <= 0) lse_stride = rows;  //                [num_parts, rows]
   switch (d) {
-    case 64: return launch_merge_d<64>(o_parts, lse_parts, num_parts, rows, o, lse, o_fp32, stream);
-    case 96: return launch_merge_d<96>(o_parts, lse_parts, num_parts, rows, o, lse, o_fp32, stream);
-    case 128: return launch_merge_d<128>(o_parts, lse_parts, num_parts, rows, o, lse, o_fp32, stream);
-    case 256: return launch_merge_d<256>(o_parts, lse_parts, num_parts, rows, o, lse, o_fp32, stream);
+    case 64: return launch_merge_d<64>(o_parts, lse_parts, num_parts, rows, o_stride, lse_stride, o, lse, o_fp32, stream);
+    case 96: return launch_merge_d<96>(o_parts, lse_parts, num_parts, rows, o_stride, lse_stride, o, lse, o_fp32, stream);
+    case 128: return launch_merge_d<128>(o_parts, lse_parts, num_parts, rows, o_stride, lse_stride, o, lse, o_fp32, stream);
+    case 256: return launch_merge_d<256>(o_parts, lse_parts, num_parts, rows, o_stride, lse_stride, o, lse, o_fp32, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -15,8 +15,10 @@ Softmax Hesaplama", applied to whole key ranges — exact in real arithmetic.
 The causal mask stays the full sequence's (bottom-right aligned): a rank
 passes the number of keys held by the ranks after it as ``kv_tail``.
 
-The exchange is two all-gathers (O and LSE) of B*Hq*Nq*(d+1) fp32 values
-per rank in all.
+The exchange is one all-gather: each rank's O and LSE are written into one
+packed buffer (O, then LSE, padded to a multiple of 4 floats), so
+B*Hq*Nq*(d+1) fp32 values per rank cross the interconnect in a single
+collective, and the merge reads the gathered parts in place.
 """
 from __future__ import annotations
 
@@ -44,9 +46,6 @@ def attention_kv_sharded(q, k_shard, v_shard, n_keys: int, causal: bool = False,
     import torch
     import torch.distributed as dist
 
-    from . import attn_fwd_partial, merge_partials
-    partial_fn = partial_fn or attn_fwd_partial
-    merge_fn = merge_fn or merge_partials
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
     if n_keys < world:
@@ -54,9 +53,23 @@ def attention_kv_sharded(q, k_shard, v_shard, n_keys: int, causal: bool = False,
     lo, hi = shard_bounds(n_keys, world, rank)
     if k_shard.shape[2] != hi - lo or v_shard.shape != k_shard.shape:
         raise ValueError(f"rank {rank} must hold keys [{lo}, {hi}) of {n_keys}")
-    o_r, lse_r = partial_fn(q, k_shard, v_shard, causal=causal, scale=scale, kv_tail=n_keys - hi)
-    o_all = torch.empty((world, *o_r.shape), dtype=o_r.dtype, device=o_r.device)
-    lse_all = torch.empty((world, *lse_r.shape), dtype=lse_r.dtype, device=lse_r.device)
-    dist.all_gather(list(o_all.unbind(0)), o_r.contiguous(), group=group)
-    dist.all_gather(list(lse_all.unbind(0)), lse_r.contiguous(), group=group)
-    return merge_fn(o_all, lse_all)
+    B, Hq, Nq, d = q.shape
+    rows = B * Hq * Nq
+    stride = (rows * d + rows + 3) // 4 * 4  # the library's packed layout (partial_packed_floats)
+    if partial_fn is None:  # the library's fp32 partial, written straight into the packed buffer
+        from . import attn_fwd_partial
+        buf = torch.empty(stride, dtype=torch.float32, device=q.device)
+        attn_fwd_partial(q, k_shard, v_shard, causal=causal, scale=scale, kv_tail=n_keys - hi,
+                         out=buf[:rows * d].view(B, Hq, Nq, d), lse=buf[rows * d:rows * d + rows].view(B, Hq, Nq))
+    else:  # another partial (same packing, in its own dtype)
+        o_p, lse_p = partial_fn(q, k_shard, v_shard, causal=causal, scale=scale, kv_tail=n_keys - hi)
+        buf = torch.zeros(stride, dtype=o_p.dtype, device=o_p.device)
+        buf[:rows * d].copy_(o_p.reshape(-1))
+        buf[rows * d:rows * d + rows].copy_(lse_p.reshape(-1))
+    parts = torch.empty((world, stride), dtype=buf.dtype, device=buf.device)
+    dist.all_gather(list(parts.unbind(0)), buf, group=group)  # the one exchange
+    if merge_fn is None:
+        from . import merge_partials_packed
+        return merge_partials_packed(parts, B, Hq, Nq, d)
+    return merge_fn(parts[:, :rows * d].reshape(world, B, Hq, Nq, d),
+                    parts[:, rows * d:rows * d + rows].reshape(world, B, Hq, Nq))

@@ -148,6 +148,21 @@ ATTN_API attn_status_t attn_merge_partials(const float* o_parts, const float* ls
                                            float* lse, void* stream);
 
 /*
+ * attn_merge_partials_packed — the same merge over parts laid out one after
+ * another in one buffer, each part = its fp32 O [B, Hq, Nq, d] followed by its
+ * fp32 LSE [B, Hq, Nq], padded to attn_partial_packed_floats() floats (a
+ * multiple of 4, so every part starts 16-byte aligned): the layout one
+ * all-gather of every rank's partial produces, so O and LSE cross the
+ * interconnect in a single collective.
+ *   parts  device, fp32 [num_parts][attn_partial_packed_floats(B, Hq, Nq, d)]
+ *   o, lse as attn_merge_partials
+ * d = 64, 96, 128 or 256. One kernel launch; allocates nothing.
+ */
+ATTN_API long long attn_partial_packed_floats(int B, int Hq, int Nq, int d);
+ATTN_API attn_status_t attn_merge_partials_packed(const float* parts, int num_parts, int B, int Hq,
+                                                  int Nq, int d, void* o, float* lse, void* stream);
+
+/*
  * attn_fwd_splitkv — attn_fwd with the keys split into ranges that run as
  * separate CTAs of one launch, then merged: for shapes with few query rows
  * per head and many keys (prefill against a long cache), where attn_fwd's

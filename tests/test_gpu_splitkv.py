@@ -166,6 +166,33 @@ def test_splitkv_long_cache_sampled_rows():
     assert d.max() <= MAX_TOL and d.mean() <= MEAN_TOL and np.abs(lg - L).max() <= LSE_TOL
 
 
+def test_packed_merge_equals_stacked_merge():
+    """merge_partials_packed over parts packed as one all-gather lays them out
+    (O then LSE per part, padded) is bit-identical to merge_partials over the
+    same parts stacked, with a part that has -inf rows."""
+    B, Hq, Hkv, Nq, Nkv, d = 1, 4, 2, 400, 900, 128  # rows 0..99 see none of the last range
+    q, k, v = make_qkv(B, Hq, Hkv, Nq, Nkv, d, seed=13)
+    from exact_attention_134_b200.kv_shard import shard_bounds
+    parts = []
+    for r in range(3):
+        lo, hi = shard_bounds(Nkv, 3, r)
+        parts.append(attn.attn_fwd_partial(q.cuda(), k[:, :, lo:hi].contiguous().cuda(),
+                                           v[:, :, lo:hi].contiguous().cuda(), causal=True,
+                                           kv_tail=Nkv - hi))
+    o_st, l_st = attn.merge_partials(torch.stack([p[0] for p in parts]), torch.stack([p[1] for p in parts]))
+    rows = B * Hq * Nq
+    stride = attn.partial_packed_floats(B, Hq, Nq, d)
+    assert stride % 4 == 0 and stride >= rows * (d + 1)
+    packed = torch.full((3, stride), float("nan"), dtype=torch.float32, device="cuda")
+    for i, (o, l) in enumerate(parts):
+        packed[i, :rows * d] = o.reshape(-1)
+        packed[i, rows * d:rows * d + rows] = l.reshape(-1)
+    o_pk, l_pk = attn.merge_partials_packed(packed, B, Hq, Nq, d)
+    _status_ok()
+    assert torch.isinf(parts[2][1]).any()
+    assert torch.equal(o_pk, o_st) and torch.equal(l_pk, l_st)
+
+
 def test_partial_split_long_range_sampled_rows():
     """Two halves of the long-cache shape's keys (causal, the first half with the
     second as its tail), each an automatically split partial (many sub-ranges
