@@ -155,18 +155,38 @@ def test_deterministic():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-def test_no_writes_outside_outputs():
-    B, H, N, d = 1, 2, 200, 64
-    q, k, v = make_qkv(B, H, H, N, N, d, seed=8)
+@pytest.mark.parametrize("path,d,causal,N", [
+    ("fwd", 64, False, 200), ("fwd", 96, True, 333), ("fwd", 128, True, 300), ("fwd", 256, True, 130),
+    ("fwd_pair", 128, True, 100), ("q8", 128, True, 300), ("fp8", 64, False, 257),
+    ("partial_split", 128, True, 100),
+])
+def test_no_writes_outside_outputs(path, d, causal, N):
+    """Canary values around O and LSE stay untouched, and every element of O
+    and LSE is written, for each output epilogue (TMA box store, row stores at
+    d = 96 and 256, head pairs, 8-bit, split-key partial in fp32)."""
+    B, Hq, Hkv = 1, 4, 2
+    Nkv = 2000 if path == "partial_split" else N
+    q, k, v = make_qkv(B, Hq, Hkv, N, Nkv, d, seed=8 + d + N)
     pad = 4096
-    obuf = torch.full((B * H * N * d + 2 * pad,), 7.0, dtype=torch.bfloat16, device="cuda")
-    lbuf = torch.full((B * H * N + 2 * pad,), 7.0, dtype=torch.float32, device="cuda")
-    o = obuf[pad:pad + B * H * N * d].view(B, H, N, d)
-    lse = lbuf[pad:pad + B * H * N].view(B, H, N)
-    attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=False, out=o, lse=lse)
+    odt = torch.float32 if path == "partial_split" else torch.bfloat16
+    n_o, n_l = B * Hq * N * d, B * Hq * N
+    obuf = torch.full((n_o + 2 * pad,), 7.0, dtype=odt, device="cuda")
+    lbuf = torch.full((n_l + 2 * pad,), 7.0, dtype=torch.float32, device="cuda")
+    o = obuf[pad:pad + n_o].view(B, Hq, N, d)
+    lse = lbuf[pad:pad + n_l].view(B, Hq, N)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    if path in ("fwd", "fwd_pair"):
+        attn.attn_fwd(qc, kc, vc, causal=causal, out=o, lse=lse)
+    elif path in ("q8", "fp8"):
+        attn.attn_fwd_q8(qc, kc, vc, causal=causal, out=o, lse=lse,
+                         qk_format="int8" if path == "q8" else "fp8")
+    else:
+        attn.attn_fwd_partial(qc, kc, vc, causal=causal, kv_tail=50, out=o, lse=lse, num_splits=4)
     torch.cuda.synchronize()
+    assert attn.get_status()[0] == 0
     assert torch.all(obuf[:pad] == 7.0) and torch.all(obuf[-pad:] == 7.0)
     assert torch.all(lbuf[:pad] == 7.0) and torch.all(lbuf[-pad:] == 7.0)
+    assert not torch.any(o == 7.0) and not torch.any(lse == 7.0)
 
 
 def test_non_default_scale_and_stream():
